@@ -1,0 +1,346 @@
+"""Benchmark of the fused, chunked top-K forward-KL loss (forward + backward).
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+                    [--workload bf16_32k] [--chunk C]
+
+One step = one ckl_fwd_bwd call over one batch of the workload: loss, dH and dW
+for T tokens (the 32K-token case by default: T=32768, d=2880, V=201088, K=100,
+chunk 2048). Inputs are seeded synthetic draws (chunked_kl_loss_logits_b200/
+workloads.py), resident in HBM before the timed region; W alone (1.16 GB) is
+larger than the 126 MB L2, so no flush is needed between steps. The timed
+region is bracketed by a barrier and a device synchronise, timed with CUDA
+events, and the max over ranks is taken. With N GPUs every rank runs its own
+replica on its own batch (tokens are independent; no collective on the data
+path), so scaling is weak and `value` is the tokens/s of all ranks together.
+
+`--impl reference` times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the oracle is the reference of this build; it is
+a deliberately slow, obviously correct program, not a tuned baseline).
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd tokens/s & TFLOP/s (% bf16 tensor peak) at T=32K, V=201088, K=100"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of this GPU's SM clock and throttle reasons."""
+
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, bus_id: str):
+        self.bus_id = bus_id.lower()
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, smax, power, reasons = [], [], [], set()
+        for ln in self.lines:
+            c = [x.strip() for x in ln.split(",")]
+            if len(c) < 9 or c[0].lower() != self.bus_id:
+                continue
+            try:
+                sm.append(float(c[1]))
+                smax.append(float(c[2]))
+                power.append(float(c[3]))
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, c[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def bus_id_of(dev: int) -> str:
+    import torch
+    p = torch.cuda.get_device_properties(dev)
+    return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+
+
+def oracle_rate(x, w, target_s: float, steps: int = 1):
+    """Time the fp64 oracle on a sample of the workload's tokens; tokens/s per step."""
+    import oracle
+    import threadpoolctl
+    rng_rows = np.arange(w.T)
+    info = threadpoolctl.threadpool_info()
+    cores = max([i.get("num_threads", 1) for i in info] + [1])
+    t0 = time.perf_counter()
+    n0 = 8
+    oracle.sampled_rows(x["H"], x["W"], x["idx"], x["logit"], rng_rows[:n0], x["mask"], with_dW=True)
+    t_probe = time.perf_counter() - t0
+    n = int(min(4096, max(n0, n0 * target_s / max(t_probe, 1e-3))))
+    rates = []
+    for s in range(steps):
+        rows = rng_rows[(s * n) % w.T:][:n]
+        t0 = time.perf_counter()
+        oracle.sampled_rows(x["H"], x["W"], x["idx"], x["logit"], rows, x["mask"], with_dW=True)
+        rates.append(len(rows) / (time.perf_counter() - t0))
+    return rates, n, cores
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    from chunked_kl_loss_logits_b200.workloads import make_inputs
+    x = make_inputs(w)
+    per_step = 4.0
+    rates, n, cores = oracle_rate(x, w, per_step, steps=args.warmup + args.steps)
+    timed = rates[args.warmup:]
+    value = float(len(timed) / sum(1.0 / r for r in timed))  # tokens/s over the timed steps
+    ms = 1000.0 * n / value
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "d": w.d, "V": w.V, "K": w.K, "chunk": w.chunk,
+                   "step": f"{n} tokens of the workload per step (whole per-token path incl. dW share)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} tokens per step, {args.steps} timed steps"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from chunked_kl_loss_logits_b200 import ckl
+    from chunked_kl_loss_logits_b200.workloads import make_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    chunk = args.chunk or w.chunk
+    x = make_inputs(w, seed=w.seed + 7919 * rank)
+    H = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
+    W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+    idx = torch.from_numpy(x["idx"]).to(dev)
+    logit = torch.from_numpy(x["logit"]).to(dev)
+    mask = None if x["mask"] is None else torch.from_numpy(x["mask"]).to(dev)
+    h = ckl.ChunkedKL(w.V, w.d, w.K, dtype=torch.bfloat16, max_chunk=chunk, device=dev)
+    ws = h.workspace(w.T, chunk)
+    out = (torch.empty((), dtype=torch.float32, device=dev), torch.empty_like(H),
+           torch.empty((w.V, w.d), dtype=torch.float32, device=dev))
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+
+    def step():
+        h.fwd_bwd(H, W, idx, logit, mask, chunk=chunk, out=out, workspace=ws, sync=False)
+
+    for _ in range(args.warmup):
+        step()
+    h.sync_status()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    sampler = ClockSampler(bus_id_of(local_rank))
+    h.profile_enable(True, 64 + args.steps * (12 * ((w.T + chunk - 1) // chunk) + 8))
+    n_launch0 = h.launch_count()
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    launches = h.launch_count() - n_launch0
+    h.sync_status()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    stats = h.profile_collect()
+    h.profile_enable(False, 0)
+    peak_mem = torch.cuda.max_memory_allocated(dev) / 2**30
+
+    # end to end: per-step inputs from pinned host memory, loss read back, every step
+    Hh = H.cpu().pin_memory()
+    ih = idx.cpu().pin_memory()
+    lh = logit.cpu().pin_memory()
+    mh = None if mask is None else mask.cpu().pin_memory()
+    stag = (torch.empty_like(H), torch.empty_like(idx), torch.empty_like(logit),
+            None if mask is None else torch.empty_like(mask))
+    h2d = Hh.numel() * 2 + ih.numel() * 4 + lh.numel() * 4 + (0 if mh is None else mh.numel())
+    h.fwd_bwd_from_host(Hh, ih, lh, mh, stag, W, chunk, out, ws)
+    barrier()
+    torch.cuda.synchronize(dev)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        h.fwd_bwd_from_host(Hh, ih, lh, mh, stag, W, chunk, out, ws)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t2 = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t2.item())
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rates, n, cores = oracle_rate(x, w, target_s=15.0)
+        cpu = {"value": rates[0], "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} of the workload's {w.T} tokens, full per-token path "
+                         f"(lse, loss, dH row, dW share), fp64 numpy/BLAS"}
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    tokens = w.T * world * args.steps
+    value = tokens / (ms_max / 1e3)
+    step_ms = ms_max / args.steps
+    useful = 6.0 * w.T * w.V * w.d
+    executed = 8.0 * w.T * w.V * w.d
+    pk_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    pk_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    kern = sorted(stats, key=lambda s: -s["total_ms"])
+    total_k = sum(s["total_ms"] for s in kern) or 1.0
+    top = kern[0]
+    avg_ms = top["total_ms"] / top["launches"]
+    if top["flops"] > 0:
+        achieved = top["flops"] / top["launches"] / (avg_ms / 1e3) / 1e12
+        roof = {"kernel": top["name"], "bound": "tensor", "achieved": achieved, "peak": pk_sus,
+                "unit": "TFLOP/s", "frac": achieved / pk_sus, "traffic": None,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                "flops_per_launch": top["flops"] / top["launches"], "avg_launch_ms": avg_ms}
+    else:
+        achieved = top["bytes"] / top["launches"] / (avg_ms / 1e3) / 1e9
+        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        roof = {"kernel": top["name"], "bound": "hbm", "achieved": achieved, "peak": hbm,
+                "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                "peak_source": f"{peak_src} hbm_gbs", "avg_launch_ms": avg_ms}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "d": w.d, "V": w.V, "K": w.K, "chunk": chunk,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "no flush: inputs larger than L2 (W alone is 1.16 GB)"},
+        "tflops_useful": useful / (step_ms / 1e3) / 1e12,
+        "tflops_executed": executed / (step_ms / 1e3) / 1e12,
+        "frac_peak_useful": useful / (step_ms / 1e3) / 1e12 / pk_burst,
+        "frac_peak_executed": executed / (step_ms / 1e3) / 1e12 / pk_burst,
+        "peak_tflops_used": {"value": pk_burst, "source": f"{peak_src} bf16_tflops"},
+        "peak_mem_gib": peak_mem,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": w.T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "kernels": [{"name": s["name"], "launches": s["launches"],
+                     "ms_per_step": s["total_ms"] / args.steps,
+                     "share": s["total_ms"] / total_k,
+                     **({"tflops": s["flops"] / (s["total_ms"] / 1e3) / 1e12} if s["flops"] else {}),
+                     **({"gbs": s["bytes"] / (s["total_ms"] / 1e3) / 1e9}
+                        if s["bytes"] and not s["flops"] else {})}
+                    for s in kern],
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="bf16_32k")
+    ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+
+    from chunked_kl_loss_logits_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and rank == 0:
+        print(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

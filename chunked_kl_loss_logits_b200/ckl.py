@@ -1,0 +1,254 @@
+"""Python binding of libckl.so (argument marshalling only).
+
+Every step of the loss runs in the library's CUDA kernels; this module only
+allocates outputs and the workspace with PyTorch, passes raw pointers and the
+current CUDA stream, and turns status codes into exceptions. If the library has
+not been built the import of `lib()` raises: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libckl.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "ckl.h")
+
+F32, BF16 = 0, 1
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported size", 3: "workspace",
+           4: "top-K index out of range", 5: "CUDA error", 6: "device wait timed out",
+           7: "pointer misaligned"}
+
+
+class CKLError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {_STATUS.get(code, code)} (status {code})")
+        self.code = code
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double)]
+
+
+_lib = None
+_P, _I64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """Load libckl.so (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m chunked_kl_loss_logits_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "ckl_create": ([ctypes.POINTER(_P), ctypes.c_int, ctypes.c_int, _I64, _I64, _I64, _I64],
+                       ctypes.c_int),
+        "ckl_destroy": ([_P], ctypes.c_int),
+        "ckl_status_str": ([ctypes.c_int], ctypes.c_char_p),
+        "ckl_workspace_bytes": ([_P, _I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
+        "ckl_fwd_bwd": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _SZ, _P, _P],
+                        ctypes.c_int),
+        "ckl_forward": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P, _P, _P, _SZ, _P, _P],
+                        ctypes.c_int),
+        "ckl_fwd_bwd_from_host": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P, _P,
+                                   _P, _SZ, _P, _P], ctypes.c_int),
+        "ckl_sync_status": ([_P, _P], ctypes.c_int),
+        "ckl_launch_count": ([_P], ctypes.c_int64),
+        "ckl_profile_enable": ([_P, ctypes.c_int, ctypes.c_int], ctypes.c_int),
+        "ckl_profile_collect": ([_P, ctypes.POINTER(KernelStat), ctypes.c_int,
+                                 ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def header_functions() -> list:
+    """Names of the functions include/ckl.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"\b(ckl_[a-z_0-9]+)\s*\(", text)))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise CKLError(code, what)
+
+
+class ChunkedKL:
+    """A handle for one LM-head shape (V x d, K cached teacher entries) on one device."""
+
+    def __init__(self, V: int, d: int, K: int, dtype=torch.bfloat16, max_chunk: int = 8192,
+                 device=None):
+        if dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError("dtype must be torch.float32 or torch.bfloat16")
+        self.V, self.d, self.K, self.dtype, self.max_chunk = V, d, K, dtype, max_chunk
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None \
+            else torch.device(device)
+        self.device = dev
+        h = _P()
+        _check(lib().ckl_create(ctypes.byref(h), dev.index or 0,
+                                F32 if dtype == torch.float32 else BF16, V, d, K, max_chunk),
+               "ckl_create")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().ckl_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------------ helpers
+    def workspace_bytes(self, T: int, chunk: int) -> int:
+        n = _SZ()
+        _check(lib().ckl_workspace_bytes(self._h, T, chunk, ctypes.byref(n)), "ckl_workspace_bytes")
+        return n.value
+
+    def workspace(self, T: int, chunk: int) -> torch.Tensor:
+        return torch.empty(max(1, self.workspace_bytes(T, chunk)), dtype=torch.uint8,
+                           device=self.device)
+
+    def launch_count(self) -> int:
+        return int(lib().ckl_launch_count(self._h))
+
+    def profile_enable(self, on: bool = True, max_launches: int = 8192):
+        _check(lib().ckl_profile_enable(self._h, int(on), max_launches), "ckl_profile_enable")
+
+    def profile_collect(self) -> list:
+        arr = (KernelStat * 32)()
+        n = ctypes.c_int()
+        _check(lib().ckl_profile_collect(self._h, arr, 32, ctypes.byref(n)), "ckl_profile_collect")
+        return [{"name": arr[i].name.decode(), "launches": arr[i].launches,
+                 "total_ms": arr[i].total_ms, "flops": arr[i].flops, "bytes": arr[i].bytes}
+                for i in range(min(n.value, 32))]
+
+    def sync_status(self, stream=None):
+        s = stream or torch.cuda.current_stream(self.device)
+        _check(lib().ckl_sync_status(self._h, ctypes.c_void_p(s.cuda_stream)), "ckl_sync_status")
+
+    def _inputs(self, H, W, idx, logit, mask):
+        T = H.shape[0]
+        if H.dtype != self.dtype or W.dtype != self.dtype:
+            raise TypeError(f"H and W must be {self.dtype}")
+        if tuple(W.shape) != (self.V, self.d) or H.shape[1] != self.d:
+            raise ValueError("H must be T x d and W must be V x d")
+        if tuple(idx.shape) != (T, self.K) or tuple(logit.shape) != (T, self.K):
+            raise ValueError("topk_idx and topk_logit must be T x K")
+        if idx.dtype != torch.int32 or logit.dtype != torch.float32:
+            raise TypeError("topk_idx must be int32 and topk_logit float32")
+        if mask is not None and (mask.dtype != torch.uint8 or mask.numel() != T):
+            raise TypeError("mask must be a uint8 tensor of T entries")
+        for t in (H, W, idx, logit) + ((mask,) if mask is not None else ()):
+            if not t.is_contiguous() or t.device != self.device:
+                raise ValueError("inputs must be contiguous tensors on the handle's device")
+        return T
+
+    # ------------------------------------------------------------------ calls
+    def fwd_bwd(self, H, W, idx, logit, mask=None, chunk: int | None = None, out=None,
+                workspace=None, token_stats: bool = False, sync: bool = True, stream=None):
+        """Loss (0-d float32 tensor), dH (T x d, dtype), dW (V x d, float32).
+
+        With token_stats=True also returns per-token logsumexp and loss (float32, T).
+        With sync=True the call waits and raises on a device-detected error.
+        """
+        T = self._inputs(H, W, idx, logit, mask)
+        chunk = min(chunk or self.max_chunk, self.max_chunk)
+        if out is None:
+            out = (torch.empty((), dtype=torch.float32, device=self.device),
+                   torch.empty_like(H), torch.empty((self.V, self.d), dtype=torch.float32,
+                                                    device=self.device))
+        loss, dH, dW = out
+        ws = workspace if workspace is not None else self.workspace(T, chunk)
+        lse = ell = None
+        if token_stats:
+            lse = torch.empty(T, dtype=torch.float32, device=self.device)
+            ell = torch.empty(T, dtype=torch.float32, device=self.device)
+        s = stream or torch.cuda.current_stream(self.device)
+        host = ctypes.c_float() if sync else None
+        code = lib().ckl_fwd_bwd(self._h, _ptr(H), _ptr(W), _ptr(idx), _ptr(logit), _ptr(mask), T,
+                                 chunk, _ptr(loss), _ptr(dH), _ptr(dW), _ptr(lse), _ptr(ell),
+                                 _ptr(ws), ws.numel(), ctypes.c_void_p(s.cuda_stream),
+                                 ctypes.byref(host) if sync else None)
+        _check(code, "ckl_fwd_bwd")
+        return (loss, dH, dW, lse, ell) if token_stats else (loss, dH, dW)
+
+    def forward(self, H, W, idx, logit, mask=None, chunk: int | None = None, workspace=None,
+                token_stats: bool = False, sync: bool = True, stream=None):
+        """Loss only (no gradients); optionally per-token logsumexp and loss."""
+        T = self._inputs(H, W, idx, logit, mask)
+        chunk = min(chunk or self.max_chunk, self.max_chunk)
+        loss = torch.empty((), dtype=torch.float32, device=self.device)
+        ws = workspace if workspace is not None else self.workspace(T, chunk)
+        lse = ell = None
+        if token_stats:
+            lse = torch.empty(T, dtype=torch.float32, device=self.device)
+            ell = torch.empty(T, dtype=torch.float32, device=self.device)
+        s = stream or torch.cuda.current_stream(self.device)
+        host = ctypes.c_float()
+        _check(lib().ckl_forward(self._h, _ptr(H), _ptr(W), _ptr(idx), _ptr(logit), _ptr(mask), T,
+                                 chunk, _ptr(loss), _ptr(lse), _ptr(ell), _ptr(ws), ws.numel(),
+                                 ctypes.c_void_p(s.cuda_stream),
+                                 ctypes.byref(host) if sync else None), "ckl_forward")
+        return (loss, lse, ell) if token_stats else loss
+
+    def fwd_bwd_from_host(self, H_host, idx_host, logit_host, mask_host, staging, W, chunk,
+                          out, workspace, stream=None) -> float:
+        """Fused loss with the per-step inputs in (pinned) host memory; returns the loss.
+
+        `staging` = (H_dev, idx_dev, logit_dev, mask_dev or None): device buffers
+        the inputs are copied into. `out` = (loss, dH, dW) device tensors.
+        """
+        H_dev, idx_dev, logit_dev, mask_dev = staging
+        loss, dH, dW = out
+        T = H_host.shape[0]
+        s = stream or torch.cuda.current_stream(self.device)
+        host = ctypes.c_float()
+        _check(lib().ckl_fwd_bwd_from_host(
+            self._h, _ptr(H_host), _ptr(idx_host), _ptr(logit_host), _ptr(mask_host),
+            _ptr(H_dev), _ptr(idx_dev), _ptr(logit_dev), _ptr(mask_dev), _ptr(W), T, chunk,
+            _ptr(loss), _ptr(dH), _ptr(dW), _ptr(workspace), workspace.numel(),
+            ctypes.c_void_p(s.cuda_stream), ctypes.byref(host)), "ckl_fwd_bwd_from_host")
+        return host.value
+
+
+class _ChunkedKLFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, H, W, idx, logit, mask, handle, chunk):
+        loss, dH, dW = handle.fwd_bwd(H.detach(), W.detach(), idx, logit, mask, chunk=chunk,
+                                      sync=False)
+        ctx.save_for_backward(dH, dW)
+        ctx.w_dtype = W.dtype
+        return loss
+
+    @staticmethod
+    def backward(ctx, g):
+        dH, dW = ctx.saved_tensors
+        return (dH * g.to(dH.dtype), (dW * g).to(ctx.w_dtype), None, None, None, None, None)
+
+
+def chunked_kl_loss(H, W, idx, logit, mask=None, chunk=None, handle: ChunkedKL | None = None):
+    """Autograd-friendly mean top-K forward KL; the gradients come from the fused call."""
+    if handle is None:
+        handle = ChunkedKL(W.shape[0], W.shape[1], idx.shape[1], dtype=W.dtype,
+                           max_chunk=max(chunk or 4096, 1), device=W.device)
+    return _ChunkedKLFn.apply(H, W, idx, logit, mask, handle, chunk)

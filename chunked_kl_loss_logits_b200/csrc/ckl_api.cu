@@ -1,0 +1,539 @@
+// C ABI of the fused, chunked top-K forward-KL loss: argument checks, the
+// workspace plan, TMA descriptors, and the per-chunk launch sequence.
+//
+// Launch sequence of one ckl_fwd_bwd call (T tokens, `chunk` at a time), after
+// the fused variant of "Chunked KL loss, running Knowledge Distillation locally
+// in less <6GB VRAM" (README, "Full Chunked KL"):
+//   mask_count                      N = sum(mask), 1/N
+//   per chunk c (Tc tokens):
+//     gather                        teacher p, merged P, sum P log P, z at the K ids, sum P z
+//     LSE contraction               per-vocabulary-tile (max, sum exp) of z = H_c W^T
+//     combine                       lse_t, l_t, gradient multipliers
+//     GRAD contraction              G = (mask/N) M exp(z - lse)   (logits recomputed)
+//     fixup                         G at the K ids -= (mask/N) P
+//     DH contraction (+ reduce)     dH_c = G W
+//     DW contraction                dW (+)= G^T H_c
+//   loss_finalize                   loss = sum mask l / N
+// The gradient tile G is the only buffer that grows with V, and it is bounded by
+// chunk x V; everything else is O(T) or O(chunk x K).
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/ckl.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace ckl;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct ProfRec {
+  int kernel;
+  int ev;
+  double flops, bytes;
+};
+
+enum KernelId {
+  KID_MASK = 0, KID_GATHER, KID_LSE, KID_COMBINE, KID_GRAD, KID_FIXUP, KID_DH, KID_DH_REDUCE,
+  KID_DW, KID_LOSS, KID_COUNT
+};
+const char* kKernelNames[KID_COUNT] = {"mask_count", "gather_topk", "lse_gemm", "lse_combine",
+                                       "grad_gemm", "topk_fixup", "dh_gemm", "dh_reduce",
+                                       "dw_gemm", "loss_finalize"};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+struct ckl_ctx {
+  int device = 0;
+  ckl_dtype dtype = CKL_F32;
+  int64_t V = 0, d = 0, K = 0, max_chunk = 0;
+  int num_sms = 0;
+  unsigned* d_status = nullptr;  // device status word
+  unsigned* h_status = nullptr;  // pinned
+  float* h_loss = nullptr;       // pinned
+  int64_t launches = 0;
+  EncodeTiledFn encode = nullptr;
+  // profiling
+  bool prof = false;
+  std::vector<cudaEvent_t> ev;  // pairs: ev[2i], ev[2i+1]
+  int ev_used = 0;
+  std::vector<ProfRec> recs;
+};
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) return;
+    ok = (prev == dev) || cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+struct WsPlan {
+  int64_t Tc = 0;  // chunk rows planned for
+  int n_vt = 0;    // vocabulary tiles of the log-sum-exp partials
+  int64_t ldG = 0;
+  int n_split = 1; // dH contraction splits (bf16)
+  size_t off_ell = 0, off_lse = 0, off_misc = 0, off_tok = 0, off_cst = 0, off_zk = 0,
+         off_Pk = 0, off_part = 0, off_G = 0, off_dHp = 0, total = 0;
+};
+
+int pick_dh_split(int64_t Tc, int64_t d, int64_t V, int num_sms) {
+  const int64_t tiles = ((Tc + 127) / 128) * ((d + 191) / 192);
+  const int64_t n_kb = (V + 63) / 64;
+  int best = 1;
+  double best_cost = 1e300;
+  for (int s = 1; s <= 8 && s <= n_kb; ++s) {
+    const double waves = std::ceil((double)(tiles * s) / std::max(1, num_sms));
+    const double cost = waves / s + 0.01 * s;  // time per unit of tile work, plus partial traffic
+    if (cost < best_cost - 1e-9) { best_cost = cost; best = s; }
+  }
+  // Every split must own at least one 64-wide block of the vocabulary.
+  const int64_t kps = (n_kb + best - 1) / best;
+  return (int)((n_kb + kps - 1) / kps);
+}
+
+WsPlan plan(const ckl_ctx* h, int64_t T, int64_t chunk, bool backward) {
+  WsPlan p;
+  p.Tc = std::max<int64_t>(1, std::min(chunk, std::max<int64_t>(T, 1)));
+  const bool bf16 = h->dtype == CKL_BF16;
+  p.n_vt = (int)((h->V + (bf16 ? 255 : 63)) / (bf16 ? 256 : 64));
+  p.ldG = (int64_t)align_up((size_t)h->V, 8);
+  p.n_split = bf16 ? pick_dh_split(p.Tc, h->d, h->V, h->num_sms) : 1;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  p.off_misc = take(sizeof(Misc));
+  p.off_ell = take((size_t)std::max<int64_t>(T, 1) * 4);
+  p.off_lse = take((size_t)std::max<int64_t>(T, 1) * 4);
+  p.off_tok = take((size_t)p.Tc * 16);
+  p.off_cst = take((size_t)p.Tc * 16);
+  p.off_zk = take((size_t)p.Tc * h->K * 4);
+  p.off_Pk = take((size_t)p.Tc * h->K * 4);
+  p.off_part = take((size_t)p.n_vt * p.Tc * 8);
+  if (backward) {
+    p.off_G = take((size_t)p.Tc * p.ldG * (bf16 ? 2 : 4));
+    if (bf16) p.off_dHp = take((size_t)p.n_split * p.Tc * h->d * 4);
+  }
+  p.total = o;
+  return p;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows
+// `row_bytes` apart, box of box_inner x box_outer, 128-byte swizzle, zero fill
+// outside the tensor.
+bool make_map(const ckl_ctx* h, CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = h->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct Launcher {
+  ckl_ctx* h;
+  cudaStream_t s;
+  template <class F>
+  cudaError_t operator()(int kid, double flops, double bytes, F&& f) {
+    int slot = -1;
+    if (h->prof && h->ev_used * 2 + 1 < (int)h->ev.size()) {
+      slot = h->ev_used++;
+      cudaEventRecord(h->ev[2 * slot], s);
+    }
+    f();
+    cudaError_t e = cudaGetLastError();
+    if (slot >= 0) {
+      cudaEventRecord(h->ev[2 * slot + 1], s);
+      h->recs.push_back(ProfRec{kid, slot, flops, bytes});
+    }
+    h->launches++;
+    return e;
+  }
+};
+
+ckl_status check_common(const ckl_ctx* h, const void* H, const void* W, const int32_t* idx,
+                        const float* logit, int64_t T, int64_t chunk, const float* loss) {
+  if (!h) return CKL_ERR_INVALID_ARG;
+  if (T < 0 || chunk < 1 || chunk > h->max_chunk || chunk > INT32_MAX) return CKL_ERR_INVALID_ARG;
+  if (!W || !loss) return CKL_ERR_INVALID_ARG;
+  if (T > 0 && (!H || !idx || !logit)) return CKL_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || (H && !aligned(H, 16)) || (idx && !aligned(idx, 16)) ||
+      (logit && !aligned(logit, 16)) || !aligned(loss, 4))
+    return CKL_ERR_ALIGNMENT;
+  return CKL_OK;
+}
+
+ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, const float* logit,
+               const uint8_t* mask, int64_t T, int64_t chunk, float* loss, void* dH, float* dW,
+               float* tok_lse, float* tok_loss, void* ws, size_t ws_bytes, cudaStream_t s,
+               bool backward) {
+  ckl_status st = check_common(h, H, W, idx, logit, T, chunk, loss);
+  if (st != CKL_OK) return st;
+  if (backward) {
+    if (!dW || (T > 0 && !dH)) return CKL_ERR_INVALID_ARG;
+    if (!aligned(dW, 16) || (dH && !aligned(dH, 16))) return CKL_ERR_ALIGNMENT;
+  }
+  if ((tok_lse && !aligned(tok_lse, 4)) || (tok_loss && !aligned(tok_loss, 4)))
+    return CKL_ERR_ALIGNMENT;
+  const WsPlan P = plan(h, T, chunk, backward);
+  if (!ws || !aligned(ws, 256) || ws_bytes < P.total) return CKL_ERR_WORKSPACE;
+
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return CKL_ERR_CUDA;
+  cudaGetLastError();  // clear a stale error so that launch checks below are ours
+
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  ChunkBufs b;
+  b.misc = reinterpret_cast<Misc*>(base + P.off_misc);
+  b.tok = reinterpret_cast<float4*>(base + P.off_tok);
+  b.cst = reinterpret_cast<float4*>(base + P.off_cst);
+  b.zk = reinterpret_cast<float*>(base + P.off_zk);
+  b.Pk = reinterpret_cast<float*>(base + P.off_Pk);
+  b.part = reinterpret_cast<float2*>(base + P.off_part);
+  b.G = backward ? base + P.off_G : nullptr;
+  b.dHp = (backward && h->dtype == CKL_BF16) ? reinterpret_cast<float*>(base + P.off_dHp) : nullptr;
+  float* ell_all = reinterpret_cast<float*>(base + P.off_ell);
+  float* lse_all = reinterpret_cast<float*>(base + P.off_lse);
+
+  const int V = (int)h->V, d = (int)h->d, K = (int)h->K;
+  const bool bf16 = h->dtype == CKL_BF16;
+  const size_t esz = bf16 ? 2 : 4;
+  Launcher L{h, s};
+  cudaError_t err = cudaSuccess;
+  auto chk = [&](cudaError_t e) { if (e != cudaSuccess && err == cudaSuccess) err = e; };
+
+  chk(L(KID_MASK, 0, (double)T, [&] { launch_mask_count(mask, T, b.misc, s); }));
+  if (backward && T == 0) chk(cudaMemsetAsync(dW, 0, (size_t)V * d * 4, s));
+
+  for (int64_t t0 = 0; t0 < T && err == cudaSuccess; t0 += chunk) {
+    const int Tc = (int)std::min<int64_t>(chunk, T - t0);
+    const double zflops = 2.0 * Tc * (double)V * d;
+    const unsigned char* Hc = static_cast<const unsigned char*>(H) + (size_t)t0 * d * esz;
+
+    chk(L(KID_GATHER, 2.0 * Tc * K * d, (double)Tc * (K * 8.0 + d * esz + K * d * esz), [&] {
+      if (bf16)
+        launch_gather<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(H),
+                                     static_cast<const __nv_bfloat16*>(W), idx, logit, t0, Tc, d,
+                                     V, K, b, h->d_status, s);
+      else
+        launch_gather<float>(static_cast<const float*>(H), static_cast<const float*>(W), idx,
+                             logit, t0, Tc, d, V, K, b, h->d_status, s);
+    }));
+
+    TcMaps mz;
+    if (bf16) {
+      if (!make_map(h, &mz.a, Hc, d, Tc, (uint64_t)d * 2, 64, 128) ||
+          !make_map(h, &mz.b, W, d, V, (uint64_t)d * 2, 64, 256))
+        return CKL_ERR_CUDA;
+    }
+    chk(L(KID_LSE, zflops, 0, [&] {
+      if (bf16) {
+        TcLaunch p{};
+        p.kind = TcKind::LSE; p.M = Tc; p.N = V; p.n_kb = (d + 63) / 64; p.n_split = 1; p.V = V;
+        p.part = b.part; p.part_ld = Tc; p.status = h->d_status; p.num_sms = h->num_sms;
+        launch_tc(mz, p, s);
+      } else {
+        launch_simt_lse(reinterpret_cast<const float*>(Hc), static_cast<const float*>(W), Tc, V,
+                        d, b.part, s);
+      }
+    }));
+    chk(L(KID_COMBINE, 0, (double)P.n_vt * Tc * 8, [&] {
+      launch_combine(t0, Tc, P.n_vt, mask, b, lse_all, ell_all, s);
+    }));
+    if (!backward) continue;
+
+    chk(L(KID_GRAD, zflops, (double)Tc * V * esz, [&] {
+      if (bf16) {
+        TcLaunch p{};
+        p.kind = TcKind::GRAD; p.M = Tc; p.N = V; p.n_kb = (d + 63) / 64; p.n_split = 1; p.V = V;
+        p.cst = b.cst; p.G = static_cast<uint16_t*>(b.G); p.ldG = P.ldG;
+        p.status = h->d_status; p.num_sms = h->num_sms;
+        launch_tc(mz, p, s);
+      } else {
+        launch_simt_grad(reinterpret_cast<const float*>(Hc), static_cast<const float*>(W), Tc, V,
+                         d, b.cst, static_cast<float*>(b.G), P.ldG, s);
+      }
+    }));
+    chk(L(KID_FIXUP, 0, (double)Tc * K * (12.0 + esz), [&] {
+      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, P.ldG, b, s);
+      else launch_fixup<float>(idx, t0, Tc, K, V, P.ldG, b, s);
+    }));
+
+    unsigned char* dHc = static_cast<unsigned char*>(dH) + (size_t)t0 * d * esz;
+    if (bf16) {
+      TcMaps mh, mw;
+      if (!make_map(h, &mh.a, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 128) ||
+          !make_map(h, &mh.b, W, d, V, (uint64_t)d * 2, 64, 64) ||
+          !make_map(h, &mw.a, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 64) ||
+          !make_map(h, &mw.b, Hc, d, Tc, (uint64_t)d * 2, 64, 64))
+        return CKL_ERR_CUDA;
+      chk(L(KID_DH, zflops, 0, [&] {
+        TcLaunch p{};
+        p.kind = TcKind::DH; p.M = Tc; p.N = d; p.n_kb = (V + 63) / 64; p.n_split = P.n_split;
+        p.dHp = b.dHp; p.status = h->d_status; p.num_sms = h->num_sms;
+        launch_tc(mh, p, s);
+      }));
+      chk(L(KID_DH_REDUCE, 0, (double)Tc * d * (4.0 * P.n_split + 2.0), [&] {
+        launch_dh_reduce_bf16(b.dHp, P.n_split, (int64_t)Tc * d, reinterpret_cast<uint16_t*>(dHc),
+                              s);
+      }));
+      chk(L(KID_DW, zflops, 0, [&] {
+        TcLaunch p{};
+        p.kind = TcKind::DW; p.M = V; p.N = d; p.n_kb = (Tc + 63) / 64; p.n_split = 1;
+        p.dW = dW; p.first = t0 == 0; p.status = h->d_status; p.num_sms = h->num_sms;
+        launch_tc(mw, p, s);
+      }));
+    } else {
+      const float* G = static_cast<const float*>(b.G);
+      chk(L(KID_DH, zflops, 0, [&] {
+        launch_simt_gemm(G, P.ldG, 1, static_cast<const float*>(W), 1, d,
+                         reinterpret_cast<float*>(dHc), d, Tc, d, V, 0, s);
+      }));
+      chk(L(KID_DW, zflops, 0, [&] {
+        launch_simt_gemm(G, 1, P.ldG, reinterpret_cast<const float*>(Hc), 1, d, dW, d, V, d, Tc,
+                         t0 > 0, s);
+      }));
+    }
+  }
+  chk(L(KID_LOSS, 0, (double)T * 5, [&] { launch_loss_finalize(ell_all, mask, T, b.misc, loss, s); }));
+  if (T > 0 && tok_lse)
+    chk(cudaMemcpyAsync(tok_lse, lse_all, (size_t)T * 4, cudaMemcpyDeviceToDevice, s));
+  if (T > 0 && tok_loss)
+    chk(cudaMemcpyAsync(tok_loss, ell_all, (size_t)T * 4, cudaMemcpyDeviceToDevice, s));
+  if (err != cudaSuccess) {
+    std::fprintf(stderr, "ckl: CUDA error: %s\n", cudaGetErrorString(err));
+    return CKL_ERR_CUDA;
+  }
+  return CKL_OK;
+}
+
+ckl_status fold_status(unsigned dev) {
+  if (dev & ST_INDEX_RANGE) return CKL_ERR_INDEX_RANGE;
+  if (dev & ST_TIMEOUT) return CKL_ERR_TIMEOUT;
+  return CKL_OK;
+}
+
+// Copy the loss and the device status to pinned host memory, wait, clear the
+// status word.
+ckl_status sync_and_read(ckl_ctx* h, cudaStream_t s, const float* loss_dev, float* loss_host) {
+  if (loss_dev && cudaMemcpyAsync(h->h_loss, loss_dev, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return CKL_ERR_CUDA;
+  if (cudaMemcpyAsync(h->h_status, h->d_status, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemsetAsync(h->d_status, 0, 4, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+    return CKL_ERR_CUDA;
+  if (loss_host && loss_dev) *loss_host = *h->h_loss;
+  return fold_status(*h->h_status);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ckl_status_str(ckl_status s) {
+  switch (s) {
+    case CKL_OK: return "ok";
+    case CKL_ERR_INVALID_ARG: return "invalid argument";
+    case CKL_ERR_UNSUPPORTED: return "unsupported size";
+    case CKL_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case CKL_ERR_INDEX_RANGE: return "a top-K index is outside [0, V)";
+    case CKL_ERR_CUDA: return "CUDA runtime error";
+    case CKL_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case CKL_ERR_ALIGNMENT: return "pointer misaligned";
+  }
+  return "unknown status";
+}
+
+ckl_status ckl_create(ckl_handle* out, int device, ckl_dtype dtype, int64_t V, int64_t d,
+                      int64_t K, int64_t max_chunk) {
+  if (!out) return CKL_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (dtype != CKL_F32 && dtype != CKL_BF16) return CKL_ERR_INVALID_ARG;
+  if (V < 1 || d < 1 || K < 1 || max_chunk < 1 || device < 0) return CKL_ERR_INVALID_ARG;
+  if (d % 8 != 0 || K > 1024 || V > (int64_t)INT32_MAX / 2 || d > 65536 || max_chunk > INT32_MAX)
+    return CKL_ERR_UNSUPPORTED;
+  const int64_t per_warp = ((d * (dtype == CKL_BF16 ? 2 : 4) + 15) / 16) * 16 + 2 * ((K * 4 + 15) / 16) * 16;
+  if (4 * per_warp > 200 * 1024) return CKL_ERR_UNSUPPORTED;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device >= ndev) return CKL_ERR_CUDA;
+  DeviceGuard guard(device);
+  if (!guard.ok) return CKL_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return CKL_ERR_CUDA;
+  if (dtype == CKL_BF16 && prop.major != 10) return CKL_ERR_UNSUPPORTED;  // tcgen05 kernels are sm_100a
+
+  ckl_ctx* h = new ckl_ctx();
+  h->device = device;
+  h->dtype = dtype;
+  h->V = V; h->d = d; h->K = K; h->max_chunk = max_chunk;
+  h->num_sms = prop.multiProcessorCount;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn) {
+    delete h;
+    return CKL_ERR_CUDA;
+  }
+  h->encode = reinterpret_cast<EncodeTiledFn>(fn);
+  if (cudaMalloc(&h->d_status, 16) != cudaSuccess) { delete h; return CKL_ERR_CUDA; }
+  if (cudaMallocHost(&h->h_status, 16) != cudaSuccess) {
+    cudaFree(h->d_status);
+    delete h;
+    return CKL_ERR_CUDA;
+  }
+  h->h_loss = reinterpret_cast<float*>(h->h_status + 1);
+  cudaMemset(h->d_status, 0, 16);
+  if (cudaDeviceSynchronize() != cudaSuccess) { ckl_destroy(h); return CKL_ERR_CUDA; }
+  *out = h;
+  return CKL_OK;
+}
+
+ckl_status ckl_destroy(ckl_handle h) {
+  if (!h) return CKL_OK;
+  DeviceGuard guard(h->device);
+  for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+  if (h->d_status) cudaFree(h->d_status);
+  if (h->h_status) cudaFreeHost(h->h_status);
+  delete h;
+  return CKL_OK;
+}
+
+ckl_status ckl_workspace_bytes(ckl_handle h, int64_t T, int64_t chunk, size_t* bytes) {
+  if (!h || !bytes || T < 0 || chunk < 1) return CKL_ERR_INVALID_ARG;
+  *bytes = plan(h, T, chunk, true).total;
+  return CKL_OK;
+}
+
+ckl_status ckl_fwd_bwd(ckl_handle h, const void* H, const void* W, const int32_t* topk_idx,
+                       const float* topk_logit, const uint8_t* mask, int64_t T, int64_t chunk,
+                       float* loss, void* dH, float* dW, float* token_lse, float* token_loss,
+                       void* workspace, size_t workspace_bytes, void* stream, float* loss_host) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ckl_status st = run(h, H, W, topk_idx, topk_logit, mask, T, chunk, loss, dH, dW, token_lse,
+                      token_loss, workspace, workspace_bytes, s, true);
+  if (st != CKL_OK || !loss_host) return st;
+  DeviceGuard guard(h->device);
+  return sync_and_read(h, s, loss, loss_host);
+}
+
+ckl_status ckl_forward(ckl_handle h, const void* H, const void* W, const int32_t* topk_idx,
+                       const float* topk_logit, const uint8_t* mask, int64_t T, int64_t chunk,
+                       float* loss, float* token_lse, float* token_loss, void* workspace,
+                       size_t workspace_bytes, void* stream, float* loss_host) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ckl_status st = run(h, H, W, topk_idx, topk_logit, mask, T, chunk, loss, nullptr, nullptr,
+                      token_lse, token_loss, workspace, workspace_bytes, s, false);
+  if (st != CKL_OK || !loss_host) return st;
+  DeviceGuard guard(h->device);
+  return sync_and_read(h, s, loss, loss_host);
+}
+
+ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t* idx_host,
+                                 const float* logit_host, const uint8_t* mask_host, void* H_dev,
+                                 int32_t* idx_dev, float* logit_dev, uint8_t* mask_dev,
+                                 const void* W, int64_t T, int64_t chunk, float* loss, void* dH,
+                                 float* dW, void* workspace, size_t workspace_bytes, void* stream,
+                                 float* loss_host) {
+  if (!h || !loss_host || T < 0) return CKL_ERR_INVALID_ARG;
+  if (T > 0 && (!H_host || !idx_host || !logit_host || !H_dev || !idx_dev || !logit_dev))
+    return CKL_ERR_INVALID_ARG;
+  if (mask_host && !mask_dev) return CKL_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  {
+    DeviceGuard guard(h->device);
+    if (!guard.ok) return CKL_ERR_CUDA;
+    const size_t esz = h->dtype == CKL_BF16 ? 2 : 4;
+    if (T > 0) {
+      if (cudaMemcpyAsync(H_dev, H_host, (size_t)T * h->d * esz, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+          cudaMemcpyAsync(idx_dev, idx_host, (size_t)T * h->K * 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+          cudaMemcpyAsync(logit_dev, logit_host, (size_t)T * h->K * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return CKL_ERR_CUDA;
+      if (mask_host &&
+          cudaMemcpyAsync(mask_dev, mask_host, (size_t)T, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return CKL_ERR_CUDA;
+    }
+  }
+  return ckl_fwd_bwd(h, H_dev, W, idx_dev, logit_dev, mask_host ? mask_dev : nullptr, T, chunk,
+                     loss, dH, dW, nullptr, nullptr, workspace, workspace_bytes, stream, loss_host);
+}
+
+ckl_status ckl_sync_status(ckl_handle h, void* stream) {
+  if (!h) return CKL_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return CKL_ERR_CUDA;
+  return sync_and_read(h, static_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+int64_t ckl_launch_count(ckl_handle h) { return h ? h->launches : -1; }
+
+ckl_status ckl_profile_enable(ckl_handle h, int enable, int max_launches) {
+  if (!h || max_launches < 0) return CKL_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return CKL_ERR_CUDA;
+  h->prof = enable != 0;
+  if (h->prof && (int)h->ev.size() < 2 * max_launches) {
+    for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+    h->ev.assign(2 * (size_t)max_launches, nullptr);
+    for (auto& e : h->ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return CKL_ERR_CUDA;
+  }
+  h->ev_used = 0;
+  h->recs.clear();
+  return CKL_OK;
+}
+
+ckl_status ckl_profile_collect(ckl_handle h, ckl_kernel_stat* stats, int max_stats, int* n_stats) {
+  if (!h || !n_stats || (max_stats > 0 && !stats)) return CKL_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return CKL_ERR_CUDA;
+  ckl_kernel_stat acc[KID_COUNT];
+  std::memset(acc, 0, sizeof(acc));
+  for (const ProfRec& r : h->recs) {
+    if (cudaEventSynchronize(h->ev[2 * r.ev + 1]) != cudaSuccess) return CKL_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, h->ev[2 * r.ev], h->ev[2 * r.ev + 1]) != cudaSuccess)
+      return CKL_ERR_CUDA;
+    ckl_kernel_stat& a = acc[r.kernel];
+    a.launches++;
+    a.total_ms += ms;
+    a.flops += r.flops;
+    a.bytes += r.bytes;
+  }
+  int n = 0;
+  for (int k = 0; k < KID_COUNT; ++k) {
+    if (acc[k].launches == 0) continue;
+    if (n < max_stats) {
+      stats[n] = acc[k];
+      std::snprintf(stats[n].name, sizeof(stats[n].name), "%s", kKernelNames[k]);
+    }
+    ++n;
+  }
+  *n_stats = n;
+  h->ev_used = 0;
+  h->recs.clear();
+  return CKL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,335 @@
+// Memory-bound kernels of the fused top-K forward-KL loss: the sparse teacher
+// term (a warp per token gathers the student logits at the K cached ids), the
+// merge of per-vocabulary-tile log-sum-exp partials, the top-K correction of the
+// gradient tile, the split-K reduction of dH, and the mask count / loss mean.
+//
+// The per-token loss follows "Chunked KL loss, running Knowledge Distillation
+// locally in less <6GB VRAM" (README formula section):
+//   l_t = sum_{v in S} P_v log P_v - sum_{v in S} P_v z_v + M logsumexp(z)
+// where only the last term spans the vocabulary; the first two need the K
+// cached entries only.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ckl {
+
+namespace {
+
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Dot product of two 16-byte vectors of the input type.
+__device__ __forceinline__ float dot16(const uint4& a, const uint4& b, const float*) {
+  return __uint_as_float(a.x) * __uint_as_float(b.x) + __uint_as_float(a.y) * __uint_as_float(b.y) +
+         __uint_as_float(a.z) * __uint_as_float(b.z) + __uint_as_float(a.w) * __uint_as_float(b.w);
+}
+__device__ __forceinline__ float dot16(const uint4& a, const uint4& b, const __nv_bfloat16*) {
+  float s = lo_bf16(a.x) * lo_bf16(b.x);
+  s = fmaf(hi_bf16(a.x), hi_bf16(b.x), s);
+  s = fmaf(lo_bf16(a.y), lo_bf16(b.y), s);
+  s = fmaf(hi_bf16(a.y), hi_bf16(b.y), s);
+  s = fmaf(lo_bf16(a.z), lo_bf16(b.z), s);
+  s = fmaf(hi_bf16(a.z), hi_bf16(b.z), s);
+  s = fmaf(lo_bf16(a.w), lo_bf16(b.w), s);
+  s = fmaf(hi_bf16(a.w), hi_bf16(b.w), s);
+  return s;
+}
+
+constexpr int kGatherWarps = 4;
+
+// One warp per token of the chunk.
+//  1. stage the token's K ids and logits (16-byte loads when K % 4 == 0) and H row
+//  2. p = softmax(logits); M = sum p; P_k = total p of slot k's id (repeats add)
+//  3. ent = sum_k p_k log P_k
+//  4. z_k = H_t . W[id_k] for every slot, 4 rows in flight per lane
+//  5. cross = sum_k p_k z_k
+template <typename Tin>
+__global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
+    const Tin* __restrict__ H, const Tin* __restrict__ W, const int32_t* __restrict__ idx,
+    const float* __restrict__ logit, int64_t t0, int Tc, int d, int V, int K, int h_bytes,
+    int k_bytes, float4* __restrict__ tok, float* __restrict__ zk_out, float* __restrict__ Pk_out,
+    unsigned* status) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kGatherWarps + warp;
+  if (i >= Tc) return;
+  const int64_t t = t0 + i;
+  unsigned char* base = smem + (size_t)warp * (h_bytes + 2 * k_bytes);
+  uint4* sH = reinterpret_cast<uint4*>(base);
+  int* sId = reinterpret_cast<int*>(base + h_bytes);
+  float* sP = reinterpret_cast<float*>(base + h_bytes + k_bytes);
+
+  // 1. stage ids, logits (into sP for now) and the H row
+  const int32_t* idr = idx + t * K;
+  const float* lgr = logit + t * K;
+  if ((K & 3) == 0) {
+    for (int k4 = lane; k4 < (K >> 2); k4 += 32) {
+      reinterpret_cast<int4*>(sId)[k4] = __ldg(reinterpret_cast<const int4*>(idr) + k4);
+      reinterpret_cast<float4*>(sP)[k4] = __ldg(reinterpret_cast<const float4*>(lgr) + k4);
+    }
+  } else {
+    for (int k = lane; k < K; k += 32) {
+      sId[k] = __ldg(idr + k);
+      sP[k] = __ldg(lgr + k);
+    }
+  }
+  constexpr int VEC = 16 / sizeof(Tin);
+  const int nvec = d / VEC;
+  const uint4* Hr = reinterpret_cast<const uint4*>(H + t * d);
+  for (int v = lane; v < nvec; v += 32) sH[v] = __ldg(Hr + v);
+  __syncwarp();
+
+  // 2. teacher softmax over the cached logits
+  float mx = -INFINITY;
+  for (int k = lane; k < K; k += 32) mx = fmaxf(mx, sP[k]);
+  mx = warp_max(mx);
+  const bool live = mx > -INFINITY;
+  float se = 0.f;
+  for (int k = lane; k < K; k += 32) se += live ? expf(sP[k] - mx) : 0.f;
+  se = warp_sum(se);
+  __syncwarp();
+  for (int k = lane; k < K; k += 32) {
+    const float p = (live && se > 0.f) ? expf(sP[k] - mx) / se : 0.f;
+    sP[k] = p;
+    const int id = sId[k];
+    if (id < 0 || id >= V) atomicOr(status, (unsigned)ST_INDEX_RANGE);
+  }
+  __syncwarp();
+
+  // 3. merged probabilities and the teacher entropy term
+  float ent = 0.f, Msum = 0.f;
+  for (int k = lane; k < K; k += 32) {
+    const int id = sId[k];
+    const float p = sP[k];
+    float P = 0.f;
+    for (int j = 0; j < K; ++j) P += (sId[j] == id) ? sP[j] : 0.f;
+    if (p > 0.f) ent += p * logf(P);
+    Msum += p;
+    Pk_out[(int64_t)i * K + k] = P;
+  }
+  ent = warp_sum(ent);
+  Msum = warp_sum(Msum);
+
+  // 4-5. student logits at the cached ids and the cross term
+  float cross = 0.f;
+  const Tin* tag = nullptr;
+  for (int k0 = 0; k0 < K; k0 += 4) {
+    int id[4];
+    bool ok[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int k = k0 + u;
+      id[u] = k < K ? sId[k] : -1;
+      ok[u] = k < K && id[u] >= 0 && id[u] < V;
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int v = lane; v < nvec; v += 32) {
+      const uint4 h = sH[v];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (ok[u]) {
+          const uint4 w = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)id[u] * d) + v);
+          acc[u] += dot16(h, w, tag);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float z = warp_sum(acc[u]);
+      const int k = k0 + u;
+      if (k < K) {
+        const float p = sP[k];
+        if (p > 0.f) cross += p * z;
+        if (lane == 0) zk_out[(int64_t)i * K + k] = z;
+      }
+    }
+  }
+  if (lane == 0) tok[i] = make_float4(ent, cross, Msum, 0.f);
+}
+
+// One thread per token: merge the per-vocabulary-tile (max, sum) partials into
+// logsumexp(z_t), then l_t = ent - cross + M lse, and the gradient multipliers.
+__global__ void combine_kernel(int64_t t0, int Tc, int n_vt, const uint8_t* __restrict__ mask,
+                               const float2* __restrict__ part, const float4* __restrict__ tok,
+                               const Misc* __restrict__ misc, float4* __restrict__ cst,
+                               float* __restrict__ lse_all, float* __restrict__ ell_all) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= Tc) return;
+  float m2 = -INFINITY;
+  for (int j = 0; j < n_vt; ++j) m2 = fmaxf(m2, part[(int64_t)j * Tc + i].x);
+  float s = 0.f;
+  for (int j = 0; j < n_vt; ++j) {
+    const float2 q = part[(int64_t)j * Tc + i];
+    s += q.y * ex2_approx(q.x - m2);
+  }
+  const float lse = (m2 + log2f(s)) * kLn2;
+  const float4 tk = tok[i];
+  const float ell = tk.x - tk.y + tk.z * lse;
+  const int64_t t = t0 + i;
+  const float sc = (mask == nullptr || mask[t] != 0) ? misc->invN : 0.f;
+  cst[i] = make_float4(lse, sc * tk.z, sc, 0.f);
+  lse_all[t] = lse;
+  ell_all[t] = ell;
+}
+
+__device__ __forceinline__ void store_g(float* G, int64_t off, float v) { G[off] = v; }
+__device__ __forceinline__ void store_g(uint16_t* G, int64_t off, float v) {
+  G[off] = f32_to_bf16(v);
+}
+
+// One thread per (token, slot): G[i][id] = gmul exp(z_k - lse) - s P_k. Slots that
+// repeat an id write the same value.
+template <typename Tg>
+__global__ void fixup_kernel(const int32_t* __restrict__ idx, int64_t t0, int Tc, int K, int V,
+                             int64_t ldG, const float4* __restrict__ cst,
+                             const float* __restrict__ zk, const float* __restrict__ Pk, Tg* G) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)Tc * K) return;
+  const int64_t i = e / K;
+  const int id = idx[t0 * K + e];
+  if (id < 0 || id >= V) return;
+  const float4 c = cst[i];
+  const float g = c.y * expf(zk[e] - c.x) - c.z * Pk[e];
+  store_g(G, i * ldG + id, g);
+}
+
+__global__ void dh_reduce_bf16_kernel(const float* __restrict__ dHp, int n_split, int64_t n_elem,
+                                      uint16_t* __restrict__ dH) {
+  const int64_t e8 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (e8 >= n_elem) return;
+  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < n_split; ++s) {
+    const float4* p = reinterpret_cast<const float4*>(dHp + s * n_elem + e8);
+    const float4 x = p[0], y = p[1];
+    a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
+    a[4] += y.x; a[5] += y.y; a[6] += y.z; a[7] += y.w;
+  }
+  uint4 o;
+  o.x = pack_bf16x2(a[0], a[1]);
+  o.y = pack_bf16x2(a[2], a[3]);
+  o.z = pack_bf16x2(a[4], a[5]);
+  o.w = pack_bf16x2(a[6], a[7]);
+  *reinterpret_cast<uint4*>(dH + e8) = o;
+}
+
+constexpr int kReduceThreads = 1024;
+
+__device__ double block_sum_d(double v, double* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  v = (threadIdx.x < (blockDim.x >> 5)) ? sh[threadIdx.x] : 0.0;
+  if (warp == 0) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  }
+  return v;  // valid in thread 0
+}
+
+// Single block: N = number of tokens with mask != 0 (all tokens when mask is NULL).
+__global__ void __launch_bounds__(kReduceThreads) mask_count_kernel(const uint8_t* mask, int64_t T,
+                                                                     Misc* misc) {
+  __shared__ double sh[32];
+  double c = 0.0;
+  if (mask == nullptr) {
+    c = threadIdx.x == 0 ? (double)T : 0.0;
+  } else {
+    long long n = 0;
+    for (int64_t t = threadIdx.x; t < T; t += blockDim.x) n += mask[t] != 0;
+    c = (double)n;
+  }
+  c = block_sum_d(c, sh);
+  if (threadIdx.x == 0) {
+    misc->N = c;
+    misc->loss_sum = 0.0;
+    misc->invN = c > 0.0 ? (float)(1.0 / c) : 0.f;
+  }
+}
+
+// Single block, fixed order: loss = sum_t mask_t l_t / N (0 when N == 0).
+__global__ void __launch_bounds__(kReduceThreads) loss_finalize_kernel(
+    const float* __restrict__ ell, const uint8_t* mask, int64_t T, Misc* misc, float* loss) {
+  __shared__ double sh[32];
+  double s = 0.0;
+  for (int64_t t = threadIdx.x; t < T; t += blockDim.x)
+    if (mask == nullptr || mask[t] != 0) s += (double)ell[t];
+  s = block_sum_d(s, sh);
+  if (threadIdx.x == 0) {
+    misc->loss_sum = s;
+    *loss = misc->N > 0.0 ? (float)(s / misc->N) : 0.f;
+  }
+}
+
+inline unsigned blocks_for(int64_t n, int per) { return (unsigned)((n + per - 1) / per); }
+
+}  // namespace
+
+void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t s) {
+  mask_count_kernel<<<1, kReduceThreads, 0, s>>>(mask, T, misc);
+}
+
+template <typename Tin>
+void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* logit, int64_t t0,
+                   int Tc, int d, int V, int K, const ChunkBufs& b, unsigned* status,
+                   cudaStream_t s) {
+  const int h_bytes = (d * (int)sizeof(Tin) + 15) & ~15;
+  const int k_bytes = (K * 4 + 15) & ~15;
+  const size_t smem = (size_t)kGatherWarps * (h_bytes + 2 * k_bytes);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(gather_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         200 * 1024);
+    attr_set = true;
+  }
+  gather_kernel<Tin><<<blocks_for(Tc, kGatherWarps), kGatherWarps * 32, smem, s>>>(
+      H, W, idx, logit, t0, Tc, d, V, K, h_bytes, k_bytes, b.tok, b.zk, b.Pk, status);
+}
+template void launch_gather<float>(const float*, const float*, const int32_t*, const float*,
+                                   int64_t, int, int, int, int, const ChunkBufs&, unsigned*,
+                                   cudaStream_t);
+template void launch_gather<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                           const int32_t*, const float*, int64_t, int, int, int,
+                                           int, const ChunkBufs&, unsigned*, cudaStream_t);
+
+void launch_combine(int64_t t0, int Tc, int n_vt, const uint8_t* mask, const ChunkBufs& b,
+                    float* lse_all, float* ell_all, cudaStream_t s) {
+  combine_kernel<<<blocks_for(Tc, 128), 128, 0, s>>>(t0, Tc, n_vt, mask, b.part, b.tok, b.misc,
+                                                      b.cst, lse_all, ell_all);
+}
+
+template <typename Tg>
+void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int64_t ldG,
+                  const ChunkBufs& b, cudaStream_t s) {
+  fixup_kernel<Tg><<<blocks_for((int64_t)Tc * K, 256), 256, 0, s>>>(
+      idx, t0, Tc, K, V, ldG, b.cst, b.zk, b.Pk, static_cast<Tg*>(b.G));
+}
+template void launch_fixup<float>(const int32_t*, int64_t, int, int, int, int64_t,
+                                  const ChunkBufs&, cudaStream_t);
+template void launch_fixup<uint16_t>(const int32_t*, int64_t, int, int, int, int64_t,
+                                     const ChunkBufs&, cudaStream_t);
+
+void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
+                           cudaStream_t s) {
+  dh_reduce_bf16_kernel<<<blocks_for(n_elem / 8, 256), 256, 0, s>>>(dHp, n_split, n_elem, dH);
+}
+
+void launch_loss_finalize(const float* ell_all, const uint8_t* mask, int64_t T, Misc* misc,
+                          float* loss, cudaStream_t s) {
+  loss_finalize_kernel<<<1, kReduceThreads, 0, s>>>(ell_all, mask, T, misc, loss);
+}
+
+}  // namespace ckl

@@ -1,0 +1,84 @@
+// Host-side launchers of the library's kernels (internal; not part of the C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ckl {
+
+// Per-token values of the chunk being processed, in the workspace.
+//   tok[i] = (ent_i, cross_i, M_i, 0)   from the teacher gather
+//   cst[i] = (lse_i, gmul_i, s_i, 0)    from the combine: gmul = s * M, s = mask/N
+struct Misc;
+struct ChunkBufs {
+  float4* tok;
+  float4* cst;
+  float* zk;     // Tc x K student logits at the cached ids
+  float* Pk;     // Tc x K merged teacher probability of each slot's id
+  float2* part;  // n_vt x Tc partial (max, sum) of exp over one vocabulary tile, log2 units
+  void* G;       // Tc x ldG scaled gradient of the logits (bf16 or f32)
+  float* dHp;    // split-K partials of dH (bf16 path)
+  struct Misc* misc;
+};
+
+// Call-wide scalars in the workspace.
+struct Misc {
+  double N;         // number of unmasked tokens
+  double loss_sum;  // sum of mask_t * l_t
+  float invN;       // 1 / N, or 0 when N == 0
+  float pad[3];
+};
+
+// ---- small kernels (k_small.cu)
+void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t s);
+template <typename Tin>
+void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* logit, int64_t t0,
+                   int Tc, int d, int V, int K, const ChunkBufs& b, unsigned* status,
+                   cudaStream_t s);
+void launch_combine(int64_t t0, int Tc, int n_vt, const uint8_t* mask, const ChunkBufs& b,
+                    float* lse_all, float* ell_all, cudaStream_t s);
+template <typename Tg>
+void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int64_t ldG,
+                  const ChunkBufs& b, cudaStream_t s);
+void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
+                           cudaStream_t s);
+void launch_loss_finalize(const float* ell_all, const uint8_t* mask, int64_t T, Misc* misc,
+                          float* loss, cudaStream_t s);
+
+// ---- fp32 SIMT path (k_simt.cu)
+void launch_simt_lse(const float* Hc, const float* W, int Tc, int V, int d, float2* part,
+                     cudaStream_t s);
+void launch_simt_grad(const float* Hc, const float* W, int Tc, int V, int d, const float4* cst,
+                      float* G, int64_t ldG, cudaStream_t s);
+// C[m][n] = (beta ? C[m][n] : 0) + sum_k A[m*sam + k*sak] * B[n*sbn + k*sbk]
+void launch_simt_gemm(const float* A, int64_t sam, int64_t sak, const float* B, int64_t sbn,
+                      int64_t sbk, float* C, int64_t ldc, int M, int N, int Kd, int beta,
+                      cudaStream_t s);
+constexpr int kSimtTile = 64;
+
+// ---- bf16 tcgen05 path (k_tc.cu)
+struct TcMaps {
+  CUtensorMap a, b;
+};
+enum class TcKind : int { LSE = 0, GRAD = 1, DH = 2, DW = 3 };
+struct TcLaunch {
+  TcKind kind;
+  int M, N, n_kb;  // output rows, output cols, 64-wide blocks along the contraction
+  int n_split;     // DH only: contraction splits (>= 1)
+  int V;           // LSE / GRAD: number of valid vocabulary columns
+  float2* part;    // LSE
+  int part_ld;     // LSE: rows of one vocabulary tile's partials (= Tc)
+  const float4* cst;  // GRAD
+  uint16_t* G;        // GRAD
+  int64_t ldG;        // GRAD
+  float* dHp;         // DH
+  float* dW;          // DW
+  int first;          // DW: overwrite instead of accumulate
+  unsigned* status;
+  int num_sms;
+};
+int tc_bn(TcKind k);  // output tile width of a kind
+cudaError_t launch_tc(const TcMaps& maps, const TcLaunch& p, cudaStream_t s);
+
+}  // namespace ckl

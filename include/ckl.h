@@ -1,0 +1,151 @@
+/*
+ * ckl.h -- fused, chunked top-K forward-KL distillation loss (C ABI).
+ *
+ * The operation is the "Full Chunked KL" loss of "Chunked KL loss, running
+ * Knowledge Distillation locally in less <6GB VRAM" (README: the three methods
+ * and the formula section). A student's last hidden states H (T x d) and LM-head
+ * weight W (V x d) give logits z = H W^T; a teacher is cached as its top-K
+ * logits per position (the forum post: "store only the top-100 logits"). Per token
+ *
+ *     l_t = sum_{v in S} P_v log P_v - sum_{v in S} P_v z_v + M * logsumexp(z)
+ *
+ * with S the cached ids, p = softmax of the cached logits, P_v the probability of
+ * id v (slots that repeat an id add up), M = sum p (1, or 0 when every cached
+ * logit is -inf). Only logsumexp spans the vocabulary. The loss is the mean of
+ * l_t over unmasked tokens (N = number of tokens with mask != 0; loss and
+ * gradients are 0 when N = 0). Gradients use the closed form
+ * dl_t/dz_v = M softmax(z)_v - P_v:
+ *     dH = (mask/N) G W,    dW = sum_t (mask_t/N) G_t^T H_t.
+ * The T x V logit tensor is never stored: the logits are produced tile by tile
+ * on the tensor cores for the log-normaliser, and recomputed chunk by chunk
+ * (chunk tokens at a time) for the gradient, as the README describes for the
+ * fused variant ("projects one sequence chunk at a time ... the backward pass
+ * recomputes each chunk and applies the closed-form gradient").
+ *
+ * Conventions for every entry point:
+ *  - All matrices are dense, row-major, contiguous. H is T x d, W is V x d,
+ *    topk_idx and topk_logit are T x K, mask is T bytes, dH is T x d, dW is V x d.
+ *  - "device" pointers are CUDA device memory of the handle's device; the caller
+ *    owns every buffer. The library allocates nothing during a call.
+ *  - H, W, dH have the handle's dtype (CKL_F32: float; CKL_BF16: bfloat16 bits).
+ *    dW, topk_logit, loss and the per-token outputs are float32; topk_idx is int32.
+ *  - H, W, dH, dW, topk_idx, topk_logit must be 16-byte aligned; the workspace
+ *    256-byte aligned. mask has no alignment requirement.
+ *  - stream is a cudaStream_t (NULL = legacy default stream); all work is
+ *    enqueued on it in order. A handle must not be used by two calls at once.
+ *  - Errors found on the host (bad sizes, null or misaligned pointers, a small
+ *    workspace) return before anything is enqueued. Errors found on the device
+ *    (a teacher id outside [0, V), a pipeline wait that exceeded its bound) set a
+ *    status word in the handle; the kernels skip the offending access and never
+ *    trap. The status is returned by the synchronising calls (loss_host != NULL,
+ *    ckl_sync_status). The outputs of a call that reports an error are undefined.
+ */
+#ifndef CKL_H
+#define CKL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ckl_ctx* ckl_handle;
+
+typedef enum {
+  CKL_OK = 0,
+  CKL_ERR_INVALID_ARG = 1,  /* null pointer, negative or inconsistent size */
+  CKL_ERR_UNSUPPORTED = 2,  /* a size the kernels do not handle (d % 8 != 0, K > 1024, ...) */
+  CKL_ERR_WORKSPACE = 3,    /* workspace null, misaligned or smaller than ckl_workspace_bytes */
+  CKL_ERR_INDEX_RANGE = 4,  /* device: a topk_idx entry outside [0, V) */
+  CKL_ERR_CUDA = 5,         /* a CUDA runtime call failed (no device, launch failure, ...) */
+  CKL_ERR_TIMEOUT = 6,      /* device: a pipeline wait exceeded its bound; the kernel gave up */
+  CKL_ERR_ALIGNMENT = 7     /* a pointer is not aligned as stated above */
+} ckl_status;
+
+typedef enum { CKL_F32 = 0, CKL_BF16 = 1 } ckl_dtype;
+
+/* Create a handle for one LM head shape on one device.
+ * device: CUDA ordinal. dtype: type of H, W, dH. V, d, K: vocabulary size, hidden
+ * size, cached entries per token (1 <= K <= 1024, d % 8 == 0, V >= 1).
+ * max_chunk: the largest chunk any call will use (>= 1).
+ * On success *out holds the handle (release with ckl_destroy). The handle owns
+ * a few bytes of device memory (status word, counters) and a pinned host word. */
+ckl_status ckl_create(ckl_handle* out, int device, ckl_dtype dtype, int64_t V, int64_t d,
+                      int64_t K, int64_t max_chunk);
+
+/* Release a handle and what it owns. NULL is accepted. */
+ckl_status ckl_destroy(ckl_handle h);
+
+/* Short English description of a status code (static storage). */
+const char* ckl_status_str(ckl_status s);
+
+/* Bytes of device workspace a call with T tokens and this chunk needs. The size
+ * is O(T) for per-token values plus O(chunk * V) for the gradient tile of one
+ * chunk, never O(T * V). */
+ckl_status ckl_workspace_bytes(ckl_handle h, int64_t T, int64_t chunk, size_t* bytes);
+
+/* Loss, dH and dW in one call (forward and backward fused).
+ * Inputs (device): H, W, topk_idx, topk_logit; mask may be NULL (all tokens count).
+ * T >= 0 tokens, processed `chunk` tokens at a time (1 <= chunk <= max_chunk).
+ * Outputs (device): loss (1 float), dH (T x d, overwritten), dW (V x d float32,
+ * overwritten, not accumulated). token_lse and token_loss (T floats each, device)
+ * are optional: logsumexp(z_t) and l_t per token (l_t is reported for masked
+ * tokens too; they are left out of the mean).
+ * loss_host: if non-NULL, the call waits for the stream, stores the loss there
+ * and returns the device-detected status; otherwise the call only enqueues work
+ * and returns CKL_OK once it is enqueued. */
+ckl_status ckl_fwd_bwd(ckl_handle h, const void* H, const void* W, const int32_t* topk_idx,
+                       const float* topk_logit, const uint8_t* mask, int64_t T, int64_t chunk,
+                       float* loss, void* dH, float* dW, float* token_lse, float* token_loss,
+                       void* workspace, size_t workspace_bytes, void* stream, float* loss_host);
+
+/* Forward only: the loss (and optional per-token values) without gradients, for
+ * evaluation. Same arguments and rules as ckl_fwd_bwd. */
+ckl_status ckl_forward(ckl_handle h, const void* H, const void* W, const int32_t* topk_idx,
+                       const float* topk_logit, const uint8_t* mask, int64_t T, int64_t chunk,
+                       float* loss, float* token_lse, float* token_loss, void* workspace,
+                       size_t workspace_bytes, void* stream, float* loss_host);
+
+/* ckl_fwd_bwd with the per-step inputs in HOST memory: copies H_host, idx_host,
+ * logit_host and mask_host (may be NULL) into the caller's device buffers H_dev,
+ * idx_dev, logit_dev, mask_dev with one cudaMemcpyAsync each on `stream` (host
+ * buffers should be pinned for the copies to be asynchronous), runs the fused
+ * loss, copies the loss back to *loss_host and waits for the stream. W stays on
+ * the device. Returns the device-detected status. */
+ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t* idx_host,
+                                 const float* logit_host, const uint8_t* mask_host, void* H_dev,
+                                 int32_t* idx_dev, float* logit_dev, uint8_t* mask_dev,
+                                 const void* W, int64_t T, int64_t chunk, float* loss, void* dH,
+                                 float* dW, void* workspace, size_t workspace_bytes, void* stream,
+                                 float* loss_host);
+
+/* Wait for `stream` and return the device-detected status of the calls enqueued
+ * on it since the last synchronising call (clears it). */
+ckl_status ckl_sync_status(ckl_handle h, void* stream);
+
+/* Number of kernels the handle has launched since it was created. */
+int64_t ckl_launch_count(ckl_handle h);
+
+/* Per-kernel timing. When enabled, each kernel launch is bracketed by CUDA
+ * events on the launching stream (a pool of `max_launches` event pairs is
+ * created here; launches past that are not timed). */
+ckl_status ckl_profile_enable(ckl_handle h, int enable, int max_launches);
+
+typedef struct {
+  char name[32];      /* kernel name */
+  int64_t launches;   /* timed launches */
+  double total_ms;    /* sum of event-measured durations */
+  double flops;       /* algorithmic FLOPs of those launches (tensor-core contractions) */
+  double bytes;       /* algorithmic DRAM bytes of those launches (memory-bound kernels) */
+} ckl_kernel_stat;
+
+/* Wait for the recorded events, fold them into per-kernel totals and clear the
+ * record. Fills up to max_stats entries; *n_stats receives the number of kernels. */
+ckl_status ckl_profile_collect(ckl_handle h, ckl_kernel_stat* stats, int max_stats, int* n_stats);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKL_H */

@@ -1,0 +1,38 @@
+"""Shared helpers of the GPU parity tests: upload seeded inputs, error measures."""
+import numpy as np
+import torch
+
+
+def rel_fro(a, b) -> float:
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / nb) if nb > 0 else float(np.linalg.norm(a))
+
+
+def rel(a, b) -> float:
+    return abs(float(a) - float(b)) / max(abs(float(b)), 1e-30)
+
+
+def upload(x, dtype, device="cuda"):
+    """Host arrays from workloads.make_inputs -> device tensors (bf16 values are exact)."""
+    dev = torch.device(device)
+    H = torch.from_numpy(x["H"]).to(dev).to(dtype).contiguous()
+    W = torch.from_numpy(x["W"]).to(dev).to(dtype).contiguous()
+    idx = torch.from_numpy(np.ascontiguousarray(x["idx"], dtype=np.int32)).to(dev)
+    logit = torch.from_numpy(np.ascontiguousarray(x["logit"], dtype=np.float32)).to(dev)
+    mask = None if x.get("mask") is None else torch.from_numpy(
+        np.ascontiguousarray(x["mask"], dtype=np.uint8)).to(dev)
+    return H, W, idx, logit, mask
+
+
+def f64(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+# Tolerances stated for the method's parity: fp32 inputs computed in fp32, bf16
+# inputs with fp32 accumulation against the oracle on the same bf16 values.
+TOL = {
+    "f32": {"loss": 1e-5, "grad": 1e-4},
+    "bf16": {"loss": 1e-3, "grad": 2e-2},
+}

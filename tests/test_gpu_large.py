@@ -1,0 +1,58 @@
+"""The 32K, 128K (packed) and 256K-token workloads at full size on the GPU.
+
+The oracle computes logsumexp, the per-token loss and dH rows for a seeded
+sample of 256 tokens (all of T enters N and the GPU run); the GPU's full-size
+outputs are also checked against properties that hold at any size: the loss is
+the mean of the per-token losses over unmasked tokens, masked tokens have zero
+dH rows, the columns of dW sum to ~0 (sum_v G_tv = 0 for every token), and the
+results do not depend on the chunk size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_kl_loss_logits_b200 import ckl
+from chunked_kl_loss_logits_b200.workloads import WORKLOADS, make_inputs, sample_rows
+from tests._helpers import TOL, f64, rel, rel_fro, upload
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+@pytest.mark.parametrize("name", ["bf16_32k", "bf16_128k_packed", "bf16_256k"])
+def test_large_workload(name):
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    rows = sample_rows(w.T, 256, seed=w.seed)
+    r = oracle.sampled_rows(x["H"], x["W"], x["idx"], x["logit"], rows, x["mask"])
+    del x["H"]
+    chunks = w.chunk_sweep or (w.chunk,)
+    h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=max(chunks))
+    rows_t = torch.from_numpy(rows).cuda()
+    ref = None
+    for chunk in chunks:
+        loss, dH, dW, lse, ell = h.fwd_bwd(H, W, idx, logit, mask, chunk=chunk, token_stats=True)
+        torch.cuda.synchronize()
+        e_lse = rel_fro(f64(lse[rows_t]), r["lse"])
+        e_ell = rel_fro(f64(ell[rows_t]), r["ell"])
+        e_dH = rel_fro(f64(dH[rows_t]), r["dH"])
+        print(name, chunk, f"lse {e_lse:.2e} ell {e_ell:.2e} dH {e_dH:.2e}")
+        assert e_lse <= 1e-5 and e_ell <= TOL["bf16"]["loss"] and e_dH <= TOL["bf16"]["grad"]
+        m = torch.ones_like(ell) if mask is None else mask.to(torch.float32)
+        mean = (ell.double() * m.double()).sum() / m.double().sum()
+        assert rel(loss.item(), mean.item()) <= 1e-5
+        if mask is not None:
+            masked = (mask == 0).nonzero().flatten()
+            assert dH[masked].abs().max().item() == 0.0
+        colsum = dW.double().sum(0)
+        assert (colsum.norm() / (dW.double().norm() * np.sqrt(w.V))).item() <= 1e-2
+        if ref is None:
+            ref = (loss.item(), dH.clone(), dW.clone(), lse.clone())
+        else:
+            assert rel(loss.item(), ref[0]) <= 1e-6
+            assert torch.equal(lse, ref[3])
+            assert ((dH.float() - ref[1].float()).norm() / ref[1].float().norm()).item() <= 1e-3
+            assert ((dW - ref[2]).norm() / ref[2].norm()).item() <= 1e-5
+        del loss, dH, dW, lse, ell
+    h.close()

@@ -1,0 +1,219 @@
+"""GPU path vs the fp64 oracle, element by element, through the C ABI.
+
+Sizes are small enough for the oracle to finish in seconds yet span several
+128 x 256 tensor-core tiles with ragged edges in every dimension (tokens,
+vocabulary, hidden size, K), plus the tiny fp32 workload and the 4K-token bf16
+workload in full (loss, dH and dW).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_kl_loss_logits_b200 import ckl
+from chunked_kl_loss_logits_b200.workloads import WORKLOADS, make_inputs, small_case
+from tests._helpers import TOL, f64, rel, rel_fro, upload
+
+pytestmark = pytest.mark.gpu
+
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def run_and_compare(x, dt, chunk, tol=None, strict=None):
+    """Run the fused call and the oracle on the same inputs; assert the stated bars."""
+    tol = tol or TOL[dt]
+    T, d = x["H"].shape
+    V, K = x["W"].shape[0], x["idx"].shape[1]
+    H, W, idx, logit, mask = upload(x, TORCH_DT[dt])
+    h = ckl.ChunkedKL(V, d, K, dtype=TORCH_DT[dt], max_chunk=max(chunk, 1))
+    loss, dH, dW, lse, ell = h.fwd_bwd(H, W, idx, logit, mask, chunk=chunk, token_stats=True)
+    r = oracle.fwd_bwd(x["H"], x["W"], x["idx"], x["logit"], x["mask"])
+    errs = {
+        "loss": rel(loss.item(), r["loss"]),
+        "dH": rel_fro(f64(dH), r["dH"]),
+        "dW": rel_fro(f64(dW), r["dW"]),
+        "lse": rel_fro(f64(lse), r["lse"]),
+        "ell": rel_fro(f64(ell), r["ell"]),
+    }
+    print(dt, x["H"].shape, V, K, chunk, {k: f"{v:.2e}" for k, v in errs.items()})
+    assert errs["loss"] <= tol["loss"], errs
+    assert errs["dH"] <= tol["grad"], errs
+    assert errs["dW"] <= tol["grad"], errs
+    assert errs["lse"] <= tol["loss"], errs
+    if strict:
+        for k, bound in strict.items():
+            assert errs[k] <= bound, (k, errs)
+    h.close()
+    return errs
+
+
+def test_tiny_f32_workload_full():
+    w = WORKLOADS["tiny_f32"]
+    x = make_inputs(w)
+    run_and_compare(x, "f32", w.chunk)
+
+
+@pytest.mark.parametrize("T,d,V,K,chunk", [
+    (300, 64, 1000, 16, 128),     # ragged tokens and vocabulary
+    (257, 136, 777, 12, 100),     # hidden size not a multiple of 64, chunk not of 128
+    (50, 64, 100, 7, 32),         # V smaller than one vocabulary tile, K % 4 != 0
+    (129, 2880, 3001, 100, 129),  # the headline hidden size and K, odd V
+    (384, 192, 2048, 32, 384),    # exact multiples everywhere
+])
+def test_bf16_ragged_shapes(T, d, V, K, chunk):
+    x = small_case(T, d, V, K, seed=T + d + V + K, dtype="bf16", teacher_var=3.0, ids="zipf")
+    run_and_compare(x, "bf16", chunk, strict={"lse": 2e-6, "dH": 1e-2, "dW": 1e-2})
+
+
+@pytest.mark.parametrize("T,d,V,K,chunk", [(200, 64, 700, 10, 64), (70, 128, 300, 4, 70)])
+def test_f32_ragged_shapes(T, d, V, K, chunk):
+    x = small_case(T, d, V, K, seed=3 * T + V, dtype="f32")
+    run_and_compare(x, "f32", chunk)
+
+
+def test_bf16_4k_workload_full():
+    w = WORKLOADS["bf16_4k"]
+    x = make_inputs(w)
+    run_and_compare(x, "bf16", w.chunk, strict={"dH": 1e-2, "dW": 1e-2})
+
+
+def test_masked_tokens_and_packing():
+    x = small_case(400, 64, 900, 16, seed=11, dtype="bf16", teacher_var=3.0, ids="zipf",
+                   packing=True)
+    assert x["mask"].sum() < 400
+    errs = run_and_compare(x, "bf16", 128)
+    assert errs["loss"] < 1e-3
+
+
+def test_all_masked_gives_zero():
+    x = small_case(100, 64, 500, 8, seed=12, dtype="bf16")
+    x["mask"] = np.zeros(100, dtype=np.uint8)
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(500, 64, 8, max_chunk=64)
+    loss, dH, dW = h.fwd_bwd(H, W, idx, logit, mask, chunk=64)
+    assert loss.item() == 0.0
+    assert dH.abs().max().item() == 0.0 and dW.abs().max().item() == 0.0
+
+
+def test_zero_tokens():
+    h = ckl.ChunkedKL(300, 64, 8, max_chunk=64)
+    W = torch.randn(300, 64, device="cuda").to(torch.bfloat16)
+    e = torch.empty(0, 64, device="cuda", dtype=torch.bfloat16)
+    ei = torch.empty(0, 8, device="cuda", dtype=torch.int32)
+    ef = torch.empty(0, 8, device="cuda", dtype=torch.float32)
+    loss, dH, dW = h.fwd_bwd(e, W, ei, ef, None, chunk=64)
+    assert loss.item() == 0.0 and dW.abs().max().item() == 0.0
+
+
+def test_single_entry_teacher_is_cross_entropy():
+    x = small_case(150, 64, 600, 1, seed=13, dtype="bf16")
+    run_and_compare(x, "bf16", 64)
+    H, W, idx, logit, _ = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(600, 64, 1, max_chunk=64)
+    loss = h.forward(H, W, idx, logit, chunk=64)
+    ce = torch.nn.functional.cross_entropy(H.double() @ W.double().T, idx[:, 0].long())
+    assert rel(loss.item(), ce.item()) < 1e-5
+
+
+def test_neg_inf_and_duplicate_ids():
+    x = small_case(120, 64, 400, 10, seed=14, dtype="bf16")
+    x["logit"][:, 7:] = -np.inf           # caches shorter than K
+    x["logit"][5, :] = -np.inf            # a token with no teacher mass
+    x["idx"][:, 3] = x["idx"][:, 1]       # repeated ids add up
+    run_and_compare(x, "bf16", 64)
+
+
+def test_out_of_range_index_is_reported():
+    x = small_case(64, 64, 300, 8, seed=15, dtype="bf16")
+    x["idx"][10, 2] = 300
+    x["idx"][20, 0] = -1
+    H, W, idx, logit, _ = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(300, 64, 8, max_chunk=64)
+    with pytest.raises(ckl.CKLError) as e:
+        h.fwd_bwd(H, W, idx, logit, None, chunk=64)
+    assert e.value.code == 4
+    # the handle stays usable and the status is cleared
+    x["idx"][10, 2] = 1
+    x["idx"][20, 0] = 2
+    H, W, idx, logit, _ = upload(x, torch.bfloat16)
+    h.fwd_bwd(H, W, idx, logit, None, chunk=64)
+
+
+def test_chunk_invariance():
+    x = small_case(520, 128, 1500, 16, seed=16, dtype="bf16", teacher_var=3.0, ids="zipf")
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(1500, 128, 16, max_chunk=520)
+    ref = None
+    for chunk in (520, 256, 200, 128, 64):
+        loss, dH, dW, lse, ell = h.fwd_bwd(H, W, idx, logit, mask, chunk=chunk, token_stats=True)
+        cur = (loss.item(), f64(dH), f64(dW), f64(lse), f64(ell))
+        if ref is None:
+            ref = cur
+            continue
+        assert rel(cur[0], ref[0]) <= 1e-6
+        assert np.array_equal(cur[3], ref[3]) and np.array_equal(cur[4], ref[4])
+        assert rel_fro(cur[1], ref[1]) <= 1e-3
+        assert rel_fro(cur[2], ref[2]) <= 1e-5
+
+
+def test_forward_only_matches_fused_loss():
+    x = small_case(260, 64, 1000, 16, seed=17, dtype="bf16")
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(1000, 64, 16, max_chunk=128)
+    l1, lse1, ell1 = h.forward(H, W, idx, logit, mask, chunk=128, token_stats=True)
+    l2, _, _, lse2, ell2 = h.fwd_bwd(H, W, idx, logit, mask, chunk=128, token_stats=True)
+    assert l1.item() == l2.item()
+    assert torch.equal(lse1, lse2) and torch.equal(ell1, ell2)
+
+
+def test_from_host_matches_device_call():
+    x = small_case(300, 64, 1000, 16, seed=18, dtype="bf16", packing=True)
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(1000, 64, 16, max_chunk=128)
+    loss, dH, dW = h.fwd_bwd(H, W, idx, logit, mask, chunk=128)
+    Hh, ih, lh, mh = (t.cpu().pin_memory() for t in (H, idx, logit, mask))
+    stag = tuple(torch.empty_like(t) for t in (H, idx, logit, mask))
+    out = (torch.empty((), device="cuda"), torch.empty_like(dH), torch.empty_like(dW))
+    ws = h.workspace(300, 128)
+    lv = h.fwd_bwd_from_host(Hh, ih, lh, mh, stag, W, 128, out, ws)
+    assert lv == loss.item()
+    assert torch.equal(out[1], dH) and torch.equal(out[2], dW)
+
+
+def test_autograd_function():
+    x = small_case(130, 64, 500, 8, seed=19, dtype="bf16")
+    H, W, idx, logit, _ = upload(x, torch.bfloat16)
+    Hp = H.clone().requires_grad_(True)
+    Wp = W.clone().requires_grad_(True)
+    loss = ckl.chunked_kl_loss(Hp, Wp, idx, logit, None, chunk=64)
+    (2.0 * loss).backward()
+    h = ckl.ChunkedKL(500, 64, 8, max_chunk=64)
+    l2, dH, dW = h.fwd_bwd(H, W, idx, logit, None, chunk=64)
+    assert loss.item() == l2.item()
+    assert torch.equal(Hp.grad, dH * 2.0)
+    assert torch.allclose(Wp.grad.float(), (dW * 2.0).to(torch.bfloat16).float())
+
+
+def test_workspace_is_linear_in_tokens_and_bounded_by_chunk():
+    h = ckl.ChunkedKL(201088, 2880, 100, max_chunk=8192)
+    a, b, c = (h.workspace_bytes(T, 2048) for T in (32768, 65536, 131072))
+    assert abs((c - b) - 2 * (b - a)) <= 4096
+    assert (b - a) / 32768 <= 16  # per-token growth: two float32 values (+ alignment)
+    # the chunk x V gradient tile dominates and scales with the chunk, not with T
+    assert h.workspace_bytes(32768, 4096) > h.workspace_bytes(32768, 2048)
+
+
+def test_launch_count_and_profiling():
+    x = small_case(256, 64, 1000, 16, seed=20, dtype="bf16")
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(1000, 64, 16, max_chunk=128)
+    n0 = h.launch_count()
+    h.profile_enable(True, 256)
+    h.fwd_bwd(H, W, idx, logit, mask, chunk=128)
+    stats = {s["name"]: s for s in h.profile_collect()}
+    n1 = h.launch_count()
+    # mask count + 2 chunks x (gather, lse, combine, grad, fixup, dh, dh_reduce, dw) + loss
+    assert n1 - n0 == 1 + 2 * 8 + 1
+    for k in ("lse_gemm", "grad_gemm", "dh_gemm", "dw_gemm", "gather_topk"):
+        assert stats[k]["launches"] == 2 and stats[k]["total_ms"] > 0
+    assert stats["lse_gemm"]["flops"] == pytest.approx(2 * 256 * 1000 * 64)
