@@ -2,9 +2,9 @@
 //
 // One persistent, warp-specialised kernel template serves the four products of
 // the method ("Chunked KL loss, running Knowledge Distillation locally in less
-// <6GB VRAM", README "Full Chunked KL": the forward projects one chunk at a time
-// and accumulates the log-normaliser; the backward recomputes each chunk and
-// applies the closed-form gradient):
+// <6GB VRAM", README "Full Chunked KL": the logits of a chunk exist only while
+// the normaliser is being accumulated, and are formed a second time in the
+// backward pass to build the analytic gradient):
 //   LSE : z = H_c W^T tile by tile; the epilogue keeps only each row's
 //         (max, sum of exp) over the tile's vocabulary columns.
 //   GRAD: z recomputed; the epilogue writes G = gmul * exp(z - lse) in bf16.

@@ -5,7 +5,8 @@
  * Knowledge Distillation locally in less <6GB VRAM" (README: the three methods
  * and the formula section). A student's last hidden states H (T x d) and LM-head
  * weight W (V x d) give logits z = H W^T; a teacher is cached as its top-K
- * logits per position (the forum post: "store only the top-100 logits"). Per token
+ * logits per position (the author's forum post: the cache keeps the 100 largest
+ * teacher logits of each position). Per token
  *
  *     l_t = sum_{v in S} P_v log P_v - sum_{v in S} P_v z_v + M * logsumexp(z)
  *
@@ -17,10 +18,10 @@
  * dl_t/dz_v = M softmax(z)_v - P_v:
  *     dH = (mask/N) G W,    dW = sum_t (mask_t/N) G_t^T H_t.
  * The T x V logit tensor is never stored: the logits are produced tile by tile
- * on the tensor cores for the log-normaliser, and recomputed chunk by chunk
- * (chunk tokens at a time) for the gradient, as the README describes for the
- * fused variant ("projects one sequence chunk at a time ... the backward pass
- * recomputes each chunk and applies the closed-form gradient").
+ * on the tensor cores for the log-normaliser, and formed again chunk by chunk
+ * (chunk tokens at a time) to build the analytic gradient: the README's fused
+ * variant, which folds the output projection into the loss and never keeps the
+ * logits of the whole sequence.
  *
  * Conventions for every entry point:
  *  - All matrices are dense, row-major, contiguous. H is T x d, W is V x d,

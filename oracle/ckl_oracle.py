@@ -18,11 +18,12 @@ the closed-form gradient and the reduction (the extracted text is cut at those
 formulas), so this module takes these readings:
 
   * p = softmax of the K cached teacher logits (the README and the forum post:
-    "store only the top-100 logits"); M = sum p, i.e. 1 unless every cached
+    the cache keeps each position's 100 largest teacher logits); M = sum p, i.e. 1 unless every cached
     logit is -inf, in which case p = 0, M = 0 and the token contributes nothing.
     A -inf logit gives p = 0 and 0 log 0 := 0.
   * Repeated ids within one token's K entries add their probabilities
-    (scatter-add reading of the dense teacher built by the "Full Dense KL" method).
+    (scatter-add reading of the dense teacher that the README's "Full Dense KL"
+    method rebuilds from the cache).
   * Temperature 1; no bias on the LM head.
   * The loss is the mean of l_t over unmasked tokens, N = sum(mask); if N = 0
     the loss and both gradients are 0.

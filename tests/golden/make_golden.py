@@ -3,8 +3,9 @@
 Run from the repository root: python tests/golden/make_golden.py
 The expected values come from the fp64 oracle only. Before writing, they are
 checked against PyTorch's fp64 kl_div on the dense teacher with autograd
-gradients (the "Full Dense KL" correctness baseline of "Chunked KL loss, running
-Knowledge Distillation locally in less <6GB VRAM").
+gradients (the dense-teacher method, "Full Dense KL", that the README of "Chunked
+KL loss, running Knowledge Distillation locally in less <6GB VRAM" uses as its
+reference for correctness).
 """
 import json
 import os

@@ -1,11 +1,11 @@
 """Pins of the fp64 oracle against facts it does not compute itself.
 
 The loss is the forward KL of "Chunked KL loss, running Knowledge Distillation
-locally in less <6GB VRAM" (README: all three methods evaluate the same forward KL
-against cached top-K teacher probabilities; the "Full Dense KL" method, which
-scatters the top-K probabilities into a dense teacher, is the correctness
-baseline), stated in the forum post to be mathematically equivalent to PyTorch's
-KL-divergence loss. Each test below pins the oracle to one of:
+locally in less <6GB VRAM" (README formula section: one forward KL shared by
+the three methods; the "Full Dense KL" method rebuilds a dense teacher from the
+cache and is the README's reference for correctness). The author's forum post
+says the loss equals PyTorch's KL divergence. Each test below pins the oracle to
+one of:
   * a dense reconstruction written separately (the pages' own baseline),
   * PyTorch's kl_div / cross_entropy with autograd gradients (fp64),
   * closed forms (K = 1, W = 0, a two-token vocabulary),
