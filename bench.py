@@ -175,6 +175,7 @@ def run_ours(args, w, rank, world, local_rank):
     logit = torch.from_numpy(x["logit"]).to(dev)
     mask = None if x["mask"] is None else torch.from_numpy(x["mask"]).to(dev)
     h = ckl.ChunkedKL(w.V, w.d, w.K, dtype=torch.bfloat16, max_chunk=chunk, device=dev)
+    h.set_recompute(args.recompute)
     ws = h.workspace(w.T, chunk)
     out = (torch.empty((), dtype=torch.float32, device=dev), torch.empty_like(H),
            torch.empty((w.V, w.d), dtype=torch.float32, device=dev))
@@ -279,6 +280,7 @@ def run_ours(args, w, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "T": w.T, "d": w.d, "V": w.V, "K": w.K, "chunk": chunk,
+                   "backward": "recompute logits" if args.recompute else "stored exp(z), bf16",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "no flush: inputs larger than L2 (W alone is 1.16 GB)"},
         "tflops_useful": useful / (step_ms / 1e3) / 1e12,
@@ -313,6 +315,8 @@ def main():
     ap.add_argument("--workload", default="bf16_32k")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--recompute", action="store_true",
+                    help="form the logits again in the backward instead of keeping exp(z)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)

@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
                                    _P, _SZ, _P, _P], ctypes.c_int),
         "ckl_sync_status": ([_P, _P], ctypes.c_int),
         "ckl_launch_count": ([_P], ctypes.c_int64),
+        "ckl_set_recompute": ([_P, ctypes.c_int], ctypes.c_int),
         "ckl_profile_enable": ([_P, ctypes.c_int, ctypes.c_int], ctypes.c_int),
         "ckl_profile_collect": ([_P, ctypes.POINTER(KernelStat), ctypes.c_int,
                                  ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -127,6 +128,10 @@ class ChunkedKL:
     def workspace(self, T: int, chunk: int) -> torch.Tensor:
         return torch.empty(max(1, self.workspace_bytes(T, chunk)), dtype=torch.uint8,
                            device=self.device)
+
+    def set_recompute(self, on: bool):
+        """bf16 only: form the logits again in the backward (True) or keep exp(z) (False)."""
+        _check(lib().ckl_set_recompute(self._h, int(on)), "ckl_set_recompute")
 
     def launch_count(self) -> int:
         return int(lib().ckl_launch_count(self._h))

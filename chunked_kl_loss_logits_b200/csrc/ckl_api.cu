@@ -7,14 +7,16 @@
 //   mask_count                      N = sum(mask), 1/N
 //   per chunk c (Tc tokens):
 //     gather                        teacher p, merged P, sum P log P, z at the K ids, sum P z
-//     LSE contraction               per-vocabulary-tile (max, sum exp) of z = H_c W^T
+//     LSE contraction               per-vocabulary-tile (max, sum exp) of z = H_c W^T;
+//                                   stored-exp mode also keeps e = exp(z - tile max), bf16
 //     combine                       lse_t, l_t, gradient multipliers
-//     GRAD contraction              G = (mask/N) M exp(z - lse)   (logits recomputed)
-//     fixup                         G at the K ids -= (mask/N) P
+//     stored-exp mode:  scale_e     G = e * (mask/N) M exp(tile max - lse)       (in place)
+//     recompute mode:   GRAD        G = (mask/N) M exp(z - lse), z formed again
+//     fixup                         G at the K ids: subtract (mask/N) P
 //     DH contraction (+ reduce)     dH_c = G W
-//     DW contraction                dW (+)= G^T H_c
+//     DW contraction                dW (+)= G^T H_c   (TMA reduce-add into dW)
 //   loss_finalize                   loss = sum mask l / N
-// The gradient tile G is the only buffer that grows with V, and it is bounded by
+// The gradient buffer G is the only one that grows with V, and it is bounded by
 // chunk x V; everything else is O(T) or O(chunk x K).
 #include <algorithm>
 #include <cmath>
@@ -43,12 +45,12 @@ struct ProfRec {
 };
 
 enum KernelId {
-  KID_MASK = 0, KID_GATHER, KID_LSE, KID_COMBINE, KID_GRAD, KID_FIXUP, KID_DH, KID_DH_REDUCE,
-  KID_DW, KID_LOSS, KID_COUNT
+  KID_MASK = 0, KID_GATHER, KID_LSE, KID_COMBINE, KID_GRAD, KID_SCALE, KID_FIXUP, KID_DH,
+  KID_DH_REDUCE, KID_DW, KID_LOSS, KID_COUNT
 };
 const char* kKernelNames[KID_COUNT] = {"mask_count", "gather_topk", "lse_gemm", "lse_combine",
-                                       "grad_gemm", "topk_fixup", "dh_gemm", "dh_reduce",
-                                       "dw_gemm", "loss_finalize"};
+                                       "grad_gemm", "scale_e", "topk_fixup", "dh_gemm",
+                                       "dh_reduce", "dw_gemm", "loss_finalize"};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -63,6 +65,7 @@ struct ckl_ctx {
   unsigned* h_status = nullptr;  // pinned
   float* h_loss = nullptr;       // pinned
   int64_t launches = 0;
+  int recompute = 0;  // bf16: form the logits again in the backward (1) or keep exp(z) (0)
   EncodeTiledFn encode = nullptr;
   // profiling
   bool prof = false;
@@ -137,16 +140,17 @@ WsPlan plan(const ckl_ctx* h, int64_t T, int64_t chunk, bool backward) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows
-// `row_bytes` apart, box of box_inner x box_outer, 128-byte swizzle, zero fill
-// outside the tensor.
+// 2-D tensor map (bf16, or fp32 when f32 is set): `inner` contiguous elements per
+// row, `outer` rows `row_bytes` apart, box of box_inner x box_outer, 128-byte
+// swizzle, zero fill outside the tensor (loads) / clipping (stores).
 bool make_map(const ckl_ctx* h, CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool f32 = false) {
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = h->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+  const CUresult r = h->encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                               2, const_cast<void*>(base),
                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -243,17 +247,24 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
                              logit, t0, Tc, d, V, K, b, h->d_status, s);
     }));
 
+    // bf16: z = H_c W^T on the tensor cores. Stored-exp mode also writes
+    // e = exp(z - tile max) into the gradient buffer (map c) for the backward.
+    const bool store_e = bf16 && backward && !h->recompute;
     TcMaps mz;
     if (bf16) {
       if (!make_map(h, &mz.a, Hc, d, Tc, (uint64_t)d * 2, 64, 128) ||
           !make_map(h, &mz.b, W, d, V, (uint64_t)d * 2, 64, 256))
         return CKL_ERR_CUDA;
+      if (backward && !make_map(h, &mz.c, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 32))
+        return CKL_ERR_CUDA;
+      if (!backward) mz.c = mz.a;
     }
-    chk(L(KID_LSE, zflops, 0, [&] {
+    chk(L(KID_LSE, zflops, store_e ? (double)Tc * V * 2 : 0, [&] {
       if (bf16) {
         TcLaunch p{};
         p.kind = TcKind::LSE; p.M = Tc; p.N = V; p.n_kb = (d + 63) / 64; p.n_split = 1; p.V = V;
-        p.part = b.part; p.part_ld = Tc; p.status = h->d_status; p.num_sms = h->num_sms;
+        p.part = b.part; p.part_ld = Tc; p.store_e = store_e ? 1 : 0;
+        p.status = h->d_status; p.num_sms = h->num_sms;
         launch_tc(mz, p, s);
       } else {
         launch_simt_lse(reinterpret_cast<const float*>(Hc), static_cast<const float*>(W), Tc, V,
@@ -265,21 +276,27 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     }));
     if (!backward) continue;
 
-    chk(L(KID_GRAD, zflops, (double)Tc * V * esz, [&] {
-      if (bf16) {
-        TcLaunch p{};
-        p.kind = TcKind::GRAD; p.M = Tc; p.N = V; p.n_kb = (d + 63) / 64; p.n_split = 1; p.V = V;
-        p.cst = b.cst; p.G = static_cast<uint16_t*>(b.G); p.ldG = P.ldG;
-        p.status = h->d_status; p.num_sms = h->num_sms;
-        launch_tc(mz, p, s);
-      } else {
-        launch_simt_grad(reinterpret_cast<const float*>(Hc), static_cast<const float*>(W), Tc, V,
-                         d, b.cst, static_cast<float*>(b.G), P.ldG, s);
-      }
-    }));
-    chk(L(KID_FIXUP, 0, (double)Tc * K * (12.0 + esz), [&] {
-      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, P.ldG, b, s);
-      else launch_fixup<float>(idx, t0, Tc, K, V, P.ldG, b, s);
+    if (store_e) {
+      chk(L(KID_SCALE, 0, (double)Tc * V * 4, [&] {
+        launch_scale_e(static_cast<uint16_t*>(b.G), P.ldG, Tc, V, b, s);
+      }));
+    } else {
+      chk(L(KID_GRAD, zflops, (double)Tc * V * esz, [&] {
+        if (bf16) {
+          TcLaunch p{};
+          p.kind = TcKind::GRAD; p.M = Tc; p.N = V; p.n_kb = (d + 63) / 64; p.n_split = 1; p.V = V;
+          p.cst = b.cst; p.G = static_cast<uint16_t*>(b.G); p.ldG = P.ldG;
+          p.status = h->d_status; p.num_sms = h->num_sms;
+          launch_tc(mz, p, s);
+        } else {
+          launch_simt_grad(reinterpret_cast<const float*>(Hc), static_cast<const float*>(W), Tc,
+                           V, d, b.cst, static_cast<float*>(b.G), P.ldG, s);
+        }
+      }));
+    }
+    chk(L(KID_FIXUP, 0, (double)Tc * K * (12.0 + 2 * esz), [&] {
+      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, P.ldG, b, !store_e, s);
+      else launch_fixup<float>(idx, t0, Tc, K, V, P.ldG, b, true, s);
     }));
 
     unsigned char* dHc = static_cast<unsigned char*>(dH) + (size_t)t0 * d * esz;
@@ -288,8 +305,10 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
       if (!make_map(h, &mh.a, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 128) ||
           !make_map(h, &mh.b, W, d, V, (uint64_t)d * 2, 64, 64) ||
           !make_map(h, &mw.a, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 64) ||
-          !make_map(h, &mw.b, Hc, d, Tc, (uint64_t)d * 2, 64, 64))
+          !make_map(h, &mw.b, Hc, d, Tc, (uint64_t)d * 2, 64, 64) ||
+          !make_map(h, &mw.c, dW, d, V, (uint64_t)d * 4, 32, 32, true))
         return CKL_ERR_CUDA;
+      mh.c = mh.a;
       chk(L(KID_DH, zflops, 0, [&] {
         TcLaunch p{};
         p.kind = TcKind::DH; p.M = Tc; p.N = d; p.n_kb = (V + 63) / 64; p.n_split = P.n_split;
@@ -487,6 +506,12 @@ ckl_status ckl_sync_status(ckl_handle h, void* stream) {
 }
 
 int64_t ckl_launch_count(ckl_handle h) { return h ? h->launches : -1; }
+
+ckl_status ckl_set_recompute(ckl_handle h, int recompute) {
+  if (!h) return CKL_ERR_INVALID_ARG;
+  h->recompute = recompute != 0;
+  return CKL_OK;
+}
 
 ckl_status ckl_profile_enable(ckl_handle h, int enable, int max_launches) {
   if (!h || max_launches < 0) return CKL_ERR_INVALID_ARG;

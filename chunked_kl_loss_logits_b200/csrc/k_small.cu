@@ -114,10 +114,16 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
     const int id = sId[k];
     const float p = sP[k];
     float P = 0.f;
-    for (int j = 0; j < K; ++j) P += (sId[j] == id) ? sP[j] : 0.f;
+    bool first = true;
+    for (int j = 0; j < K; ++j) {
+      if (sId[j] == id) {
+        P += sP[j];
+        first = first && (j >= k);
+      }
+    }
     if (p > 0.f) ent += p * logf(P);
     Msum += p;
-    Pk_out[(int64_t)i * K + k] = P;
+    Pk_out[(int64_t)i * K + k] = first ? P : 0.f;
   }
   ent = warp_sum(ent);
   Msum = warp_sum(Msum);
@@ -125,28 +131,43 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
   // 4-5. student logits at the cached ids and the cross term
   float cross = 0.f;
   const Tin* tag = nullptr;
-  for (int k0 = 0; k0 < K; k0 += 4) {
-    int id[4];
-    bool ok[4];
+  constexpr int R = 8;  // W rows in flight per warp
+  for (int k0 = 0; k0 < K; k0 += R) {
+    const uint4* row[R];
+    bool ok[R];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < R; ++u) {
       const int k = k0 + u;
-      id[u] = k < K ? sId[k] : -1;
-      ok[u] = k < K && id[u] >= 0 && id[u] < V;
+      const int id = k < K ? sId[k] : -1;
+      ok[u] = k < K && id >= 0 && id < V;
+      row[u] = reinterpret_cast<const uint4*>(W + (int64_t)(ok[u] ? id : 0) * d);
     }
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int v = lane; v < nvec; v += 32) {
-      const uint4 h = sH[v];
+    float acc[R];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < R; ++u) acc[u] = 0.f;
+    int v = lane;
+    for (; v + 32 < nvec; v += 64) {
+      const uint4 h0 = sH[v], h1 = sH[v + 32];
+      uint4 w0[R], w1[R];
+#pragma unroll
+      for (int u = 0; u < R; ++u) {
         if (ok[u]) {
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)id[u] * d) + v);
-          acc[u] += dot16(h, w, tag);
+          w0[u] = __ldg(row[u] + v);
+          w1[u] = __ldg(row[u] + v + 32);
         }
       }
+#pragma unroll
+      for (int u = 0; u < R; ++u)
+        if (ok[u]) acc[u] += dot16(h0, w0[u], tag) + dot16(h1, w1[u], tag);
+    }
+    if (v < nvec) {
+      const uint4 h0 = sH[v];
+#pragma unroll
+      for (int u = 0; u < R; ++u)
+        if (ok[u]) acc[u] += dot16(h0, __ldg(row[u] + v), tag);
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < R; ++u) {
       const float z = warp_sum(acc[u]);
       const int k = k0 + u;
       if (k < K) {
@@ -159,50 +180,102 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
   if (lane == 0) tok[i] = make_float4(ent, cross, Msum, 0.f);
 }
 
-// One thread per token: merge the per-vocabulary-tile (max, sum) partials into
-// logsumexp(z_t), then l_t = ent - cross + M lse, and the gradient multipliers.
-__global__ void combine_kernel(int64_t t0, int Tc, int n_vt, const uint8_t* __restrict__ mask,
-                               const float2* __restrict__ part, const float4* __restrict__ tok,
-                               const Misc* __restrict__ misc, float4* __restrict__ cst,
-                               float* __restrict__ lse_all, float* __restrict__ ell_all) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= Tc) return;
-  float m2 = -INFINITY;
-  for (int j = 0; j < n_vt; ++j) m2 = fmaxf(m2, part[(int64_t)j * Tc + i].x);
-  float s = 0.f;
-  for (int j = 0; j < n_vt; ++j) {
-    const float2 q = part[(int64_t)j * Tc + i];
-    s += q.y * ex2_approx(q.x - m2);
+constexpr int kCombTok = 32, kCombSplit = 8;
+
+// Merge the per-vocabulary-tile (max, sum) partials into logsumexp(z_t), then
+// l_t = ent - cross + M lse and the gradient multipliers. A block covers 32
+// tokens; its 8 warps each merge every 8th vocabulary tile (coalesced 256-byte
+// reads of 32 consecutive tokens), then one warp merges the 8 results.
+__global__ void __launch_bounds__(kCombTok * kCombSplit) combine_kernel(
+    int64_t t0, int Tc, int n_vt, const uint8_t* __restrict__ mask,
+    const float2* __restrict__ part, const float4* __restrict__ tok, const Misc* __restrict__ misc,
+    float4* __restrict__ cst, float* __restrict__ lse_all, float* __restrict__ ell_all) {
+  __shared__ float sm[kCombSplit][kCombTok], ss[kCombSplit][kCombTok];
+  const int tk = threadIdx.x % kCombTok, sp = threadIdx.x / kCombTok;
+  const int i = blockIdx.x * kCombTok + tk;
+  float m2 = -INFINITY, s = 0.f;
+  if (i < Tc) {
+#pragma unroll 4
+    for (int j = sp; j < n_vt; j += kCombSplit) {
+      const float2 q = part[(int64_t)j * Tc + i];
+      if (q.x > m2) {
+        s = s * ex2_approx(m2 - q.x) + q.y;
+        m2 = q.x;
+      } else {
+        s += q.y * ex2_approx(q.x - m2);
+      }
+    }
   }
-  const float lse = (m2 + log2f(s)) * kLn2;
-  const float4 tk = tok[i];
-  const float ell = tk.x - tk.y + tk.z * lse;
+  sm[sp][tk] = m2;
+  ss[sp][tk] = s;
+  __syncthreads();
+  if (sp != 0 || i >= Tc) return;
+  float M2 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kCombSplit; ++j) M2 = fmaxf(M2, sm[j][tk]);
+  float S = 0.f;
+#pragma unroll
+  for (int j = 0; j < kCombSplit; ++j)
+    if (sm[j][tk] > -INFINITY) S += ss[j][tk] * ex2_approx(sm[j][tk] - M2);
+  const float lse = (M2 + log2f(S)) * kLn2;
+  const float4 t4 = tok[i];
+  const float ell = t4.x - t4.y + t4.z * lse;
   const int64_t t = t0 + i;
   const float sc = (mask == nullptr || mask[t] != 0) ? misc->invN : 0.f;
-  cst[i] = make_float4(lse, sc * tk.z, sc, 0.f);
+  cst[i] = make_float4(lse, sc * t4.z, sc, 0.f);
   lse_all[t] = lse;
   ell_all[t] = ell;
+}
+
+// Stored-exp forward: the gradient buffer holds e = exp2(z log2e - m2_tile) in
+// bf16; turn it into G = gmul exp(z - lse) = e * gmul * exp2(m2_tile - lse log2e)
+// in place. A thread handles 8 consecutive columns of one row.
+__global__ void scale_e_kernel(uint16_t* __restrict__ G, int64_t ldG, int Tc, int V,
+                               const float2* __restrict__ part, const float4* __restrict__ cst) {
+  const int n8 = (V + 7) / 8;
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)Tc * n8) return;
+  const int i = (int)(e / n8);
+  const int c8 = (int)(e - (int64_t)i * n8) * 8;
+  const float4 c = cst[i];
+  const float m2 = part[(int64_t)(c8 >> 8) * Tc + i].x;
+  const float f = c.y * ex2_approx(m2 - c.x * 1.4426950408889634f);
+  uint4* p = reinterpret_cast<uint4*>(G + (int64_t)i * ldG + c8);
+  uint4 x = *p;
+  x.x = pack_bf16x2(lo_bf16(x.x) * f, hi_bf16(x.x) * f);
+  x.y = pack_bf16x2(lo_bf16(x.y) * f, hi_bf16(x.y) * f);
+  x.z = pack_bf16x2(lo_bf16(x.z) * f, hi_bf16(x.z) * f);
+  x.w = pack_bf16x2(lo_bf16(x.w) * f, hi_bf16(x.w) * f);
+  *p = x;
 }
 
 __device__ __forceinline__ void store_g(float* G, int64_t off, float v) { G[off] = v; }
 __device__ __forceinline__ void store_g(uint16_t* G, int64_t off, float v) {
   G[off] = f32_to_bf16(v);
 }
+__device__ __forceinline__ float load_g(const float* G, int64_t off) { return G[off]; }
+__device__ __forceinline__ float load_g(const uint16_t* G, int64_t off) {
+  return bf16_to_f32(G[off]);
+}
 
-// One thread per (token, slot): G[i][id] = gmul exp(z_k - lse) - s P_k. Slots that
-// repeat an id write the same value.
+// One thread per (token, slot) that holds the first occurrence of an id (P_k > 0):
+// overwrite: G[i][id] = gmul exp(z_k - lse) - s P_k;  else: G[i][id] -= s P_k.
 template <typename Tg>
 __global__ void fixup_kernel(const int32_t* __restrict__ idx, int64_t t0, int Tc, int K, int V,
                              int64_t ldG, const float4* __restrict__ cst,
-                             const float* __restrict__ zk, const float* __restrict__ Pk, Tg* G) {
+                             const float* __restrict__ zk, const float* __restrict__ Pk, Tg* G,
+                             int overwrite) {
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= (int64_t)Tc * K) return;
+  const float P = Pk[e];
+  if (!(P > 0.f)) return;
   const int64_t i = e / K;
   const int id = idx[t0 * K + e];
   if (id < 0 || id >= V) return;
   const float4 c = cst[i];
-  const float g = c.y * expf(zk[e] - c.x) - c.z * Pk[e];
-  store_g(G, i * ldG + id, g);
+  const int64_t off = i * ldG + id;
+  const float g = overwrite ? c.y * expf(zk[e] - c.x) - c.z * P : load_g(G, off) - c.z * P;
+  store_g(G, off, g);
 }
 
 __global__ void dh_reduce_bf16_kernel(const float* __restrict__ dHp, int n_split, int64_t n_elem,
@@ -307,20 +380,25 @@ template void launch_gather<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bflo
 
 void launch_combine(int64_t t0, int Tc, int n_vt, const uint8_t* mask, const ChunkBufs& b,
                     float* lse_all, float* ell_all, cudaStream_t s) {
-  combine_kernel<<<blocks_for(Tc, 128), 128, 0, s>>>(t0, Tc, n_vt, mask, b.part, b.tok, b.misc,
-                                                      b.cst, lse_all, ell_all);
+  combine_kernel<<<blocks_for(Tc, kCombTok), kCombTok * kCombSplit, 0, s>>>(
+      t0, Tc, n_vt, mask, b.part, b.tok, b.misc, b.cst, lse_all, ell_all);
+}
+
+void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s) {
+  scale_e_kernel<<<blocks_for((int64_t)Tc * ((V + 7) / 8), 256), 256, 0, s>>>(G, ldG, Tc, V,
+                                                                            b.part, b.cst);
 }
 
 template <typename Tg>
 void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int64_t ldG,
-                  const ChunkBufs& b, cudaStream_t s) {
+                  const ChunkBufs& b, bool overwrite, cudaStream_t s) {
   fixup_kernel<Tg><<<blocks_for((int64_t)Tc * K, 256), 256, 0, s>>>(
-      idx, t0, Tc, K, V, ldG, b.cst, b.zk, b.Pk, static_cast<Tg*>(b.G));
+      idx, t0, Tc, K, V, ldG, b.cst, b.zk, b.Pk, static_cast<Tg*>(b.G), overwrite ? 1 : 0);
 }
 template void launch_fixup<float>(const int32_t*, int64_t, int, int, int, int64_t,
-                                  const ChunkBufs&, cudaStream_t);
+                                  const ChunkBufs&, bool, cudaStream_t);
 template void launch_fixup<uint16_t>(const int32_t*, int64_t, int, int, int, int64_t,
-                                     const ChunkBufs&, cudaStream_t);
+                                     const ChunkBufs&, bool, cudaStream_t);
 
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
                            cudaStream_t s) {

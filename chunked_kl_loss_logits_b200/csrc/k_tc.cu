@@ -1,16 +1,19 @@
 // bf16 tensor-core contractions of the fused top-K forward-KL loss on sm_100a.
 //
-// One persistent, warp-specialised kernel template serves the four products of
-// the method ("Chunked KL loss, running Knowledge Distillation locally in less
-// <6GB VRAM", README "Full Chunked KL": the logits of a chunk exist only while
-// the normaliser is being accumulated, and are formed a second time in the
-// backward pass to build the analytic gradient):
-//   LSE : z = H_c W^T tile by tile; the epilogue keeps only each row's
-//         (max, sum of exp) over the tile's vocabulary columns.
-//   GRAD: z recomputed; the epilogue writes G = gmul * exp(z - lse) in bf16.
-//   DH  : dH_c = G W, contraction over the vocabulary split in n_split ranges
-//         (fp32 partials, reduced in a fixed order afterwards).
-//   DW  : dW (+)= G^T H_c, contraction over the chunk's tokens.
+// One persistent, warp-specialised kernel template serves the products of the
+// method ("Chunked KL loss, running Knowledge Distillation locally in less <6GB
+// VRAM", README "Full Chunked KL": the logits of a chunk exist only while the
+// normaliser is being accumulated, and the backward pass needs the analytic
+// gradient of each chunk):
+//   LSE : z = H_c W^T tile by tile; the epilogue keeps each row's (max, sum of
+//         exp) over the tile's vocabulary columns. With `store_e` it also writes
+//         e = exp(z - tile max) in bf16 to the chunk's gradient buffer, so the
+//         backward pass can rescale it instead of forming z again.
+//   GRAD: z formed again; the epilogue writes G = gmul * exp(z - lse) in bf16.
+//   DH  : dH_c = G W, the vocabulary split in n_split ranges (fp32 partials,
+//         reduced in a fixed order afterwards).
+//   DW  : dW (+)= G^T H_c, contraction over the chunk's tokens; the epilogue adds
+//         its fp32 tile into dW with a TMA reduce-add (the add happens in L2).
 //
 // CTA layout (192 threads, one CTA per SM):
 //   warp 0      TMA producer: 128B-swizzled tiles of A and B into a STAGES-deep
@@ -19,7 +22,8 @@
 //               (M=128, N=BN, K=16) into one of two TMEM accumulators and
 //               commits each stage back to the producer.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (thread = output row),
-//               then the kind's math and global stores, overlapped with the MMA
+//               the kind's math, then either plain stores or 128B-swizzled
+//               shared-memory staging + TMA bulk stores, overlapped with the MMA
 //               of the next tile through the second accumulator.
 // Operand layouts: H, W and G are read K-major for LSE/GRAD/DH-A; W (DH-B), G
 // (DW-A) and H (DW-B) are read MN-major, so no operand is ever transposed in
@@ -32,19 +36,20 @@ namespace ckl {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BK = 64;               // 64 bf16 = one 128-byte swizzle row
+constexpr int BK = 64;                // 64 bf16 = one 128-byte swizzle row
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
-constexpr int kAccStride = 256;      // TMEM columns between the two accumulators
-constexpr int kAtomBytes = 64 * 128; // one 64 (MN) x 64 (K) MN-major box
+constexpr int kAccStride = 256;       // TMEM columns between the two accumulators
+constexpr int kAtomBytes = 64 * 128;  // one 64 (MN) x 64 (K) MN-major box
+constexpr int kStageBufBytes = 4096;  // one epilogue staging box: 32 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <TcKind KIND>
 struct Cfg;
-template <> struct Cfg<TcKind::LSE>  { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 4; };
-template <> struct Cfg<TcKind::GRAD> { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 4; };
-template <> struct Cfg<TcKind::DH>   { static constexpr int BN = 192; static constexpr bool A_MN = false, B_MN = true;  static constexpr int STAGES = 5; };
-template <> struct Cfg<TcKind::DW>   { static constexpr int BN = 192; static constexpr bool A_MN = true,  B_MN = true;  static constexpr int STAGES = 5; };
+template <> struct Cfg<TcKind::LSE>  { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 4; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::GRAD> { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 4; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::DH>   { static constexpr int BN = 192; static constexpr bool A_MN = false, B_MN = true;  static constexpr int STAGES = 5; static constexpr bool STAGED = false; };
+template <> struct Cfg<TcKind::DW>   { static constexpr int BN = 192; static constexpr bool A_MN = true,  B_MN = true;  static constexpr int STAGES = 4; static constexpr bool STAGED = true; };
 
 template <TcKind KIND>
 struct Layout {
@@ -54,8 +59,11 @@ struct Layout {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  // two staging boxes per epilogue warp
+  static constexpr int EPI_BYTES = Cfg<KIND>::STAGED ? 4 * 2 * kStageBufBytes : 0;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + RING_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + RING_BYTES + EPI_BYTES + BAR_BYTES;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
 struct TileCoord {
@@ -80,10 +88,35 @@ __device__ __forceinline__ TileCoord tile_coord(const TcLaunch& p, int n_m, int 
   return c;
 }
 
+// Write one thread's 128-byte row (8 x 16 bytes) into a 32-row staging box laid
+// out as the 128-byte TMA swizzle expects: 16-byte chunk c of row r sits at
+// position c ^ (r % 8).
+__device__ __forceinline__ void stage_row(unsigned char* box, int r, const uint4 (&chunks)[8]) {
+  uint4* rowp = reinterpret_cast<uint4*>(box + r * 128);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) rowp[c ^ (r & 7)] = chunks[c];
+}
+
+// Pack 32 + 32 fp32 values as 64 bf16 (one staged row of a 64-column box).
+__device__ __forceinline__ void pack_row_bf16(const float (&a)[32], const float (&b)[32],
+                                              uint4 (&out)[8]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    out[c] = make_uint4(pack_bf16x2(a[8 * c], a[8 * c + 1]), pack_bf16x2(a[8 * c + 2], a[8 * c + 3]),
+                        pack_bf16x2(a[8 * c + 4], a[8 * c + 5]),
+                        pack_bf16x2(a[8 * c + 6], a[8 * c + 7]));
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    out[4 + c] = make_uint4(pack_bf16x2(b[8 * c], b[8 * c + 1]),
+                            pack_bf16x2(b[8 * c + 2], b[8 * c + 3]),
+                            pack_bf16x2(b[8 * c + 4], b[8 * c + 5]),
+                            pack_bf16x2(b[8 * c + 6], b[8 * c + 7]));
+}
+
 template <TcKind KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const TcLaunch p) {
+              const __grid_constant__ CUtensorMap tmC, const TcLaunch p) {
   using L = Layout<KIND>;
   constexpr int BN = L::BN;
   constexpr int STAGES = L::STAGES;
@@ -92,7 +125,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::RING_BYTES);
+  unsigned char* epi_smem = smem + L::RING_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::RING_BYTES + L::EPI_BYTES);
   uint64_t* full = bars;                 // [STAGES]
   uint64_t* empty = bars + STAGES;       // [STAGES]
   uint64_t* tfull = bars + 2 * STAGES;   // [2]
@@ -124,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (Cfg<KIND>::STAGED) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -220,6 +255,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;   // accumulator row owned by this thread
+    unsigned char* stg = epi_smem + q * 2 * kStageBufBytes;  // this warp's two staging boxes
+    int nstage = 0;                  // staging boxes this warp has filled so far
+    // Fill staging box (nstage & 1) from this thread's row and hand it to TMA.
+    auto stage_and_issue = [&](const uint4 (&chunks)[8], int c0, int c1, bool reduce) {
+      if (c1 >= p.M) return;  // every row of this warp's box lies past the tensor (warp-uniform)
+      unsigned char* box = stg + (nstage & 1) * kStageBufBytes;
+      if (lane == 0) bulk_wait_read<1>();  // the box's previous store has read it
+      __syncwarp();
+      stage_row(box, lane, chunks);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (reduce) tma_reduce_add_2d(&tmC, box, c0, c1);
+        else tma_store_2d(&tmC, box, c0, c1);
+        bulk_commit();
+      }
+      ++nstage;
+    };
+
     int it = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       const TileCoord c = tile_coord(p, n_m, n_n, kps, tile);
@@ -231,27 +285,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int grow = c.mt * BM + row;  // output row (token for LSE/GRAD/DH, vocab id for DW)
       const bool row_ok = grow < p.M;
       const int col0 = c.nt * BN;
+      const int row0 = c.mt * BM + q * 32;  // first row of this warp's staging boxes
 
       if constexpr (KIND == TcKind::LSE) {
-        float m2 = -INFINITY, s = 0.f;
+        // (max, sum exp2) over the tile's valid columns, in log2 units.
+        float m2 = -INFINITY;
 #pragma unroll 1
         for (int cc = 0; cc < BN / 32; ++cc) {
           float v[32];
           tmem_ld32(taddr + cc * 32, v);
           const int cb = col0 + cc * 32;
-          float cm = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            v[j] = (cb + j < p.V) ? v[j] * kLog2e : -INFINITY;
-            cm = fmaxf(cm, v[j]);
-          }
-          if (cm > m2) {
-            if (m2 > -INFINITY) s *= ex2_approx(m2 - cm);
-            m2 = cm;
-          }
-          if (m2 > -INFINITY) {
+          for (int j = 0; j < 32; ++j)
+            if (cb + j < p.V) m2 = fmaxf(m2, v[j] * kLog2e);
+        }
+        float s = 0.f;
+        if (!p.store_e) {
+#pragma unroll 1
+          for (int cc = 0; cc < BN / 32; ++cc) {
+            float v[32];
+            tmem_ld32(taddr + cc * 32, v);
+            const int cb = col0 + cc * 32;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) s += ex2_approx(v[j] - m2);
+            for (int j = 0; j < 32; ++j)
+              s += (cb + j < p.V) ? ex2_approx(fmaf(v[j], kLog2e, -m2)) : 0.f;
+          }
+        } else {
+          // e = exp2(z log2e - m2) in (0, 1], stored as bf16 64 columns at a time
+#pragma unroll 1
+          for (int cc = 0; cc < BN / 64; ++cc) {
+            float a[32], b[32];
+            tmem_ld32(taddr + cc * 64, a);
+            tmem_ld32(taddr + cc * 64 + 32, b);
+            const int cb = col0 + cc * 64;
+            // same expressions and summation order (column by column) as above,
+            // so lse does not depend on whether e is stored
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              a[j] = (cb + j < p.V) ? ex2_approx(fmaf(a[j], kLog2e, -m2)) : 0.f;
+              s += a[j];
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              b[j] = (cb + 32 + j < p.V) ? ex2_approx(fmaf(b[j], kLog2e, -m2)) : 0.f;
+              s += b[j];
+            }
+            if (cb < p.V) {
+              uint4 ch[8];
+              pack_row_bf16(a, b, ch);
+              stage_and_issue(ch, cb, row0, false);
+            }
           }
         }
         if (row_ok) p.part[(int64_t)c.nt * p.part_ld + grow] = make_float2(m2, s);
@@ -262,35 +345,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           lse2 = cs.x * kLog2e;
           gmul = cs.y;
         }
-        uint16_t* grow_ptr = p.G + (int64_t)grow * p.ldG;
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          float v[32];
-          tmem_ld32(taddr + cc * 32, v);
-          const int cb = col0 + cc * 32;
-          if (!row_ok || cb >= p.V) continue;
-          uint32_t pk[16];
+        for (int cc = 0; cc < BN / 64; ++cc) {
+          float a[32], b[32];
+          tmem_ld32(taddr + cc * 64, a);
+          tmem_ld32(taddr + cc * 64 + 32, b);
+          const int cb = col0 + cc * 64;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            pk[j] = pack_bf16x2(gmul * ex2_approx(fmaf(v[2 * j], kLog2e, -lse2)),
-                                gmul * ex2_approx(fmaf(v[2 * j + 1], kLog2e, -lse2)));
-          if (cb + 32 <= p.V) {
-            uint4* dst = reinterpret_cast<uint4*>(grow_ptr + cb);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (cb + j < p.V)
-                grow_ptr[cb + j] = (uint16_t)((j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu));
+          for (int j = 0; j < 32; ++j) {
+            a[j] = gmul * ex2_approx(fmaf(a[j], kLog2e, -lse2));
+            b[j] = gmul * ex2_approx(fmaf(b[j], kLog2e, -lse2));
+          }
+          if (cb < p.V) {
+            uint4 ch[8];
+            pack_row_bf16(a, b, ch);
+            stage_and_issue(ch, cb, row0, false);
           }
         }
-      } else {
-        // DH: fp32 partial of split c.split; DW: dW (+)= acc.
-        float* out = (KIND == TcKind::DH)
-                         ? p.dHp + (int64_t)c.split * p.M * p.N + (int64_t)grow * p.N
-                         : p.dW + (int64_t)grow * p.N;
+      } else if constexpr (KIND == TcKind::DH) {
+        // fp32 partial of split c.split, plain vector stores
+        float* out = p.dHp + (int64_t)c.split * p.M * p.N + (int64_t)grow * p.N;
 #pragma unroll 1
         for (int cc = 0; cc < BN / 32; ++cc) {
           float v[32];
@@ -299,29 +373,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!row_ok || cb >= p.N) continue;
           if (cb + 32 <= p.N) {
             float4* dst = reinterpret_cast<float4*>(out + cb);
-            if (KIND == TcKind::DW && !p.first) {
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                float4 o = dst[j];
-                o.x += v[4 * j]; o.y += v[4 * j + 1]; o.z += v[4 * j + 2]; o.w += v[4 * j + 3];
-                dst[j] = o;
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            }
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (cb + j < p.N)
-                out[cb + j] = (KIND == TcKind::DW && !p.first) ? out[cb + j] + v[j] : v[j];
+              if (cb + j < p.N) out[cb + j] = v[j];
           }
+        }
+      } else {
+        // DW: stage 32 fp32 columns per box and add them into dW in L2
+        // (store instead of add for the first chunk).
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          float v[32];
+          tmem_ld32(taddr + cc * 32, v);
+          const int cb = col0 + cc * 32;
+          if (cb >= p.N) continue;
+          uint4 ch[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            ch[j] = make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                               __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+          stage_and_issue(ch, cb, row0, !p.first);
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
     }
+    if (Cfg<KIND>::STAGED && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -343,7 +424,7 @@ cudaError_t launch_kind(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
                                        L::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = n_tiles < p.num_sms ? n_tiles : p.num_sms;
-  tc_kernel<KIND><<<grid, kThreads, L::SMEM_BYTES, s>>>(maps.a, maps.b, p);
+  tc_kernel<KIND><<<grid, kThreads, L::SMEM_BYTES, s>>>(maps.a, maps.b, maps.c, p);
   return cudaGetLastError();
 }
 

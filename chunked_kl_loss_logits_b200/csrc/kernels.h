@@ -15,7 +15,8 @@ struct ChunkBufs {
   float4* tok;
   float4* cst;
   float* zk;     // Tc x K student logits at the cached ids
-  float* Pk;     // Tc x K merged teacher probability of each slot's id
+  float* Pk;     // Tc x K total teacher probability of each slot's id; 0 on every slot
+                 // but the first that holds a given id (so each id is corrected once)
   float2* part;  // n_vt x Tc partial (max, sum) of exp over one vocabulary tile, log2 units
   void* G;       // Tc x ldG scaled gradient of the logits (bf16 or f32)
   float* dHp;    // split-K partials of dH (bf16 path)
@@ -38,9 +39,13 @@ void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* 
                    cudaStream_t s);
 void launch_combine(int64_t t0, int Tc, int n_vt, const uint8_t* mask, const ChunkBufs& b,
                     float* lse_all, float* ell_all, cudaStream_t s);
+// G at the cached ids. overwrite: G = gmul exp(z_k - lse) - s P_k (the gradient
+// contraction wrote gmul exp(z - lse) there); otherwise G -= s P_k in place.
 template <typename Tg>
 void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int64_t ldG,
-                  const ChunkBufs& b, cudaStream_t s);
+                  const ChunkBufs& b, bool overwrite, cudaStream_t s);
+// Stored-exp forward: G[i][v] = e[i][v] * gmul_i * exp2(m2[tile(v)][i] - lse_i log2 e), in place.
+void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s);
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
                            cudaStream_t s);
 void launch_loss_finalize(const float* ell_all, const uint8_t* mask, int64_t T, Misc* misc,
@@ -59,7 +64,7 @@ constexpr int kSimtTile = 64;
 
 // ---- bf16 tcgen05 path (k_tc.cu)
 struct TcMaps {
-  CUtensorMap a, b;
+  CUtensorMap a, b, c;  // operands A and B; c = epilogue store target (G or dW)
 };
 enum class TcKind : int { LSE = 0, GRAD = 1, DH = 2, DW = 3 };
 struct TcLaunch {
@@ -69,6 +74,7 @@ struct TcLaunch {
   int V;           // LSE / GRAD: number of valid vocabulary columns
   float2* part;    // LSE
   int part_ld;     // LSE: rows of one vocabulary tile's partials (= Tc)
+  int store_e;     // LSE: also store exp(z - tile max) in bf16 through map c
   const float4* cst;  // GRAD
   uint16_t* G;        // GRAD
   int64_t ldG;        // GRAD

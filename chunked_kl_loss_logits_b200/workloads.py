@@ -69,6 +69,10 @@ WORKLOADS = {
                                  "zipf", packing=True, seed=1004),
     "bf16_256k": Workload("bf16_256k", 262144, 2880, 201088, 100, 2048, "bf16", 3.0, "zipf",
                           chunk_sweep=(512, 1024, 2048, 4096, 8192), seed=1005),
+    # Profiling case: one 2048-token chunk of the headline shapes (d, K, chunk) with
+    # a 32000-word vocabulary, so W (184 MB) still exceeds L2 while the whole
+    # footprint stays under 1 GB for multi-pass counter captures.
+    "prof_2k": Workload("prof_2k", 2048, 2880, 32000, 100, 2048, "bf16", 3.0, "zipf", seed=1099),
 }
 
 _STREAMS = ("perm", "ids", "logits", "H", "W", "mask")

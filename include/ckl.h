@@ -125,6 +125,15 @@ ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t
  * on it since the last synchronising call (clears it). */
 ckl_status ckl_sync_status(ckl_handle h, void* stream);
 
+/* bf16 handles only: choose how the backward pass obtains exp(z - lse).
+ * recompute = 1: the logits are formed a second time on the tensor cores from H
+ * and W, as the README's fused variant does (executed work 8 T V d).
+ * recompute = 0 (default): the forward contraction also writes exp(z - tile max)
+ * in bf16 into the chunk x V gradient buffer, and the backward rescales it in
+ * place (executed work 6 T V d plus one 4-byte pass over the buffer). Memory is
+ * the same in both modes. fp32 handles always recompute. */
+ckl_status ckl_set_recompute(ckl_handle h, int recompute);
+
 /* Number of kernels the handle has launched since it was created. */
 int64_t ckl_launch_count(ckl_handle h);
 

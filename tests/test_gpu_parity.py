@@ -19,13 +19,14 @@ pytestmark = pytest.mark.gpu
 TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 
-def run_and_compare(x, dt, chunk, tol=None, strict=None):
+def run_and_compare(x, dt, chunk, tol=None, strict=None, recompute=False):
     """Run the fused call and the oracle on the same inputs; assert the stated bars."""
     tol = tol or TOL[dt]
     T, d = x["H"].shape
     V, K = x["W"].shape[0], x["idx"].shape[1]
     H, W, idx, logit, mask = upload(x, TORCH_DT[dt])
     h = ckl.ChunkedKL(V, d, K, dtype=TORCH_DT[dt], max_chunk=max(chunk, 1))
+    h.set_recompute(recompute)
     loss, dH, dW, lse, ell = h.fwd_bwd(H, W, idx, logit, mask, chunk=chunk, token_stats=True)
     r = oracle.fwd_bwd(x["H"], x["W"], x["idx"], x["logit"], x["mask"])
     errs = {
@@ -35,7 +36,8 @@ def run_and_compare(x, dt, chunk, tol=None, strict=None):
         "lse": rel_fro(f64(lse), r["lse"]),
         "ell": rel_fro(f64(ell), r["ell"]),
     }
-    print(dt, x["H"].shape, V, K, chunk, {k: f"{v:.2e}" for k, v in errs.items()})
+    print(dt, "recompute" if recompute else "stored", x["H"].shape, V, K, chunk,
+          {k: f"{v:.2e}" for k, v in errs.items()})
     assert errs["loss"] <= tol["loss"], errs
     assert errs["dH"] <= tol["grad"], errs
     assert errs["dW"] <= tol["grad"], errs
@@ -60,9 +62,11 @@ def test_tiny_f32_workload_full():
     (129, 2880, 3001, 100, 129),  # the headline hidden size and K, odd V
     (384, 192, 2048, 32, 384),    # exact multiples everywhere
 ])
-def test_bf16_ragged_shapes(T, d, V, K, chunk):
+@pytest.mark.parametrize("recompute", [False, True], ids=["stored", "recompute"])
+def test_bf16_ragged_shapes(T, d, V, K, chunk, recompute):
     x = small_case(T, d, V, K, seed=T + d + V + K, dtype="bf16", teacher_var=3.0, ids="zipf")
-    run_and_compare(x, "bf16", chunk, strict={"lse": 2e-6, "dH": 1e-2, "dW": 1e-2})
+    run_and_compare(x, "bf16", chunk, strict={"lse": 2e-6, "dH": 1e-2, "dW": 1e-2},
+                    recompute=recompute)
 
 
 @pytest.mark.parametrize("T,d,V,K,chunk", [(200, 64, 700, 10, 64), (70, 128, 300, 4, 70)])
@@ -71,10 +75,11 @@ def test_f32_ragged_shapes(T, d, V, K, chunk):
     run_and_compare(x, "f32", chunk)
 
 
-def test_bf16_4k_workload_full():
+@pytest.mark.parametrize("recompute", [False, True], ids=["stored", "recompute"])
+def test_bf16_4k_workload_full(recompute):
     w = WORKLOADS["bf16_4k"]
     x = make_inputs(w)
-    run_and_compare(x, "bf16", w.chunk, strict={"dH": 1e-2, "dW": 1e-2})
+    run_and_compare(x, "bf16", w.chunk, strict={"dH": 1e-2, "dW": 1e-2}, recompute=recompute)
 
 
 def test_masked_tokens_and_packing():
@@ -115,12 +120,26 @@ def test_single_entry_teacher_is_cross_entropy():
     assert rel(loss.item(), ce.item()) < 1e-5
 
 
-def test_neg_inf_and_duplicate_ids():
+@pytest.mark.parametrize("recompute", [False, True], ids=["stored", "recompute"])
+def test_neg_inf_and_duplicate_ids(recompute):
     x = small_case(120, 64, 400, 10, seed=14, dtype="bf16")
     x["logit"][:, 7:] = -np.inf           # caches shorter than K
     x["logit"][5, :] = -np.inf            # a token with no teacher mass
     x["idx"][:, 3] = x["idx"][:, 1]       # repeated ids add up
-    run_and_compare(x, "bf16", 64)
+    x["idx"][:, 8] = x["idx"][:, 1]       # ... also on a slot with zero probability
+    run_and_compare(x, "bf16", 64, recompute=recompute)
+
+
+def test_backward_modes_agree():
+    x = small_case(300, 128, 1200, 16, seed=21, dtype="bf16", teacher_var=3.0, ids="zipf")
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(1200, 128, 16, max_chunk=128)
+    h.set_recompute(False)
+    l0, dH0, dW0 = (t.clone() for t in h.fwd_bwd(H, W, idx, logit, mask, chunk=128))
+    h.set_recompute(True)
+    l1, dH1, dW1 = h.fwd_bwd(H, W, idx, logit, mask, chunk=128)
+    assert l0.item() == l1.item()
+    assert rel_fro(f64(dH0), f64(dH1)) <= 1e-2 and rel_fro(f64(dW0), f64(dW1)) <= 1e-2
 
 
 def test_out_of_range_index_is_reported():
@@ -212,8 +231,8 @@ def test_launch_count_and_profiling():
     h.fwd_bwd(H, W, idx, logit, mask, chunk=128)
     stats = {s["name"]: s for s in h.profile_collect()}
     n1 = h.launch_count()
-    # mask count + 2 chunks x (gather, lse, combine, grad, fixup, dh, dh_reduce, dw) + loss
+    # mask count + 2 chunks x (gather, lse, combine, scale_e, fixup, dh, dh_reduce, dw) + loss
     assert n1 - n0 == 1 + 2 * 8 + 1
-    for k in ("lse_gemm", "grad_gemm", "dh_gemm", "dw_gemm", "gather_topk"):
+    for k in ("lse_gemm", "scale_e", "dh_gemm", "dw_gemm", "gather_topk"):
         assert stats[k]["launches"] == 2 and stats[k]["total_ms"] > 0
     assert stats["lse_gemm"]["flops"] == pytest.approx(2 * 256 * 1000 * 64)
