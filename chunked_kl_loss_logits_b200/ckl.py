@@ -257,3 +257,33 @@ def chunked_kl_loss(H, W, idx, logit, mask=None, chunk=None, handle: ChunkedKL |
         handle = ChunkedKL(W.shape[0], W.shape[1], idx.shape[1], dtype=W.dtype,
                            max_chunk=max(chunk or 4096, 1), device=W.device)
     return _ChunkedKLFn.apply(H, W, idx, logit, mask, handle, chunk)
+
+
+def forward_static(H, W, idx, logit, mask=None, chunk: int = 2048, stream=None,
+                   token_stats: bool = False):
+    """Forward-only loss through ckl_forward_static: no device allocation by the library.
+
+    For callers that may not allocate device memory: the library's scratch is a
+    fixed 32 MiB device array shared by all calls (overlapping calls race). The
+    outputs here are allocated by torch on the caller's side; pass your own
+    buffers to the C entry point if that is not allowed either. Returns the loss
+    (0-d float32 tensor), plus per-token logsumexp and loss when token_stats.
+    """
+    f = lib().ckl_forward_static
+    f.argtypes = [ctypes.c_int, ctypes.c_int, _I64, _I64, _I64, _P, _P, _P, _P, _P, _I64, _I64,
+                  _P, _P, _P, _P, _P]
+    f.restype = ctypes.c_int
+    T, d = H.shape
+    V, K = W.shape[0], idx.shape[1]
+    dev = H.device
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse = ell = None
+    if token_stats:
+        lse = torch.empty(T, dtype=torch.float32, device=dev)
+        ell = torch.empty(T, dtype=torch.float32, device=dev)
+    s = stream or torch.cuda.current_stream(dev)
+    host = ctypes.c_float()
+    _check(f(dev.index or 0, F32 if H.dtype == torch.float32 else BF16, V, d, K, _ptr(H), _ptr(W),
+             _ptr(idx), _ptr(logit), _ptr(mask), T, chunk, _ptr(loss), _ptr(lse), _ptr(ell),
+             ctypes.c_void_p(s.cuda_stream), ctypes.byref(host)), "ckl_forward_static")
+    return (loss, lse, ell) if token_stats else loss

@@ -562,3 +562,114 @@ ckl_status ckl_profile_collect(ckl_handle h, ckl_kernel_stat* stats, int max_sta
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward-only loss without any device allocation.
+//
+// Some callers cannot call cudaMalloc: code embedded in a runtime that owns all
+// device memory through its own arena or caching allocator (and forbids outside
+// allocations), and latency-critical loops that cannot afford the device-wide
+// synchronisation cudaMalloc / cudaFree imply. ckl_create allocates (a status
+// word, a pinned host word), so this entry point takes no handle: its scratch
+// (the status word plus the forward workspace) lives in one file-scope device
+// array of kStaticScratchBytes that every GPU loading this library holds until
+// the process exits. Calls share the array, so calls that overlap on the GPU
+// (two streams, or two host threads) race and must be serialised by the caller.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
+constexpr size_t kStaticStatusBytes = 256;                // status word, then the workspace
+constexpr int kStaticMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+struct StaticDevice {
+  bool ready = false;
+  unsigned char* scratch = nullptr;  // device address of g_static_scratch on this device
+  int num_sms = 0;
+  int cc_major = 0;
+  EncodeTiledFn encode = nullptr;
+};
+std::mutex g_static_mu;
+StaticDevice g_static_dev[kStaticMaxDevices];
+
+// Once per device, with that device current: the device address of the static
+// array (the host-side symbol is only a stand-in), the SM count and the TMA
+// descriptor encoder.
+ckl_status static_setup(int device, StaticDevice** out) {
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  StaticDevice& sd = g_static_dev[device];
+  if (!sd.ready) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return CKL_ERR_CUDA;
+    int sms = 0, major = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess)
+      return CKL_ERR_CUDA;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return CKL_ERR_CUDA;
+    sd.scratch = static_cast<unsigned char*>(ptr);
+    sd.num_sms = sms;
+    sd.cc_major = major;
+    sd.encode = reinterpret_cast<EncodeTiledFn>(fn);
+    sd.ready = true;
+  }
+  *out = &sd;
+  return CKL_OK;
+}
+
+}  // namespace
+
+extern "C" ckl_status ckl_forward_static(int device, ckl_dtype dtype, int64_t V, int64_t d,
+                                         int64_t K, const void* H, const void* W,
+                                         const int32_t* topk_idx, const float* topk_logit,
+                                         const uint8_t* mask, int64_t T, int64_t chunk,
+                                         float* loss, float* token_lse, float* token_loss,
+                                         void* stream, float* loss_host) {
+  if (dtype != CKL_F32 && dtype != CKL_BF16) return CKL_ERR_INVALID_ARG;
+  if (V < 1 || d < 1 || K < 1 || chunk < 1 || T < 0 || device < 0 || device >= kStaticMaxDevices)
+    return CKL_ERR_INVALID_ARG;
+  if (d % 8 != 0 || K > 1024 || V > (int64_t)INT32_MAX / 2 || d > 65536 || chunk > INT32_MAX)
+    return CKL_ERR_UNSUPPORTED;
+  const int64_t per_warp =
+      ((d * (dtype == CKL_BF16 ? 2 : 4) + 15) / 16) * 16 + 2 * ((K * 4 + 15) / 16) * 16;
+  if (4 * per_warp > 200 * 1024) return CKL_ERR_UNSUPPORTED;
+  DeviceGuard guard(device);
+  if (!guard.ok) return CKL_ERR_CUDA;
+  StaticDevice* sd = nullptr;
+  ckl_status st = static_setup(device, &sd);
+  if (st != CKL_OK) return st;
+  if (dtype == CKL_BF16 && sd->cc_major != 10) return CKL_ERR_UNSUPPORTED;
+
+  // A handle-shaped view of this call; it owns nothing.
+  ckl_ctx c;
+  c.device = device;
+  c.dtype = dtype;
+  c.V = V; c.d = d; c.K = K; c.max_chunk = chunk;
+  c.num_sms = sd->num_sms;
+  c.encode = sd->encode;
+  c.d_status = reinterpret_cast<unsigned*>(sd->scratch);
+  const WsPlan P = plan(&c, T, chunk, false);
+  if (P.total > kStaticScratchBytes - kStaticStatusBytes) return CKL_ERR_WORKSPACE;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The status word must start at zero; every workspace piece the forward pass
+  // reads is written earlier in the same call.
+  if (cudaMemsetAsync(c.d_status, 0, sizeof(unsigned), s) != cudaSuccess) return CKL_ERR_CUDA;
+  st = run(&c, H, W, topk_idx, topk_logit, mask, T, chunk, loss, nullptr, nullptr, token_lse,
+           token_loss, sd->scratch + kStaticStatusBytes, kStaticScratchBytes - kStaticStatusBytes,
+           s, false);
+  if (st != CKL_OK || !loss_host) return st;
+  unsigned dev_status = 0;
+  float host_loss = 0.f;
+  if (cudaMemcpyAsync(&host_loss, loss, sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(&dev_status, c.d_status, sizeof(unsigned), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return CKL_ERR_CUDA;
+  *loss_host = host_loss;
+  return fold_status(dev_status);
+}

@@ -121,6 +121,32 @@ ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t
                                  float* dW, void* workspace, size_t workspace_bytes, void* stream,
                                  float* loss_host);
 
+/* Forward-only loss that allocates nothing, for callers that may not call
+ * cudaMalloc: code embedded in a runtime that owns all device memory through its
+ * own arena or caching allocator, and latency-critical loops that cannot afford
+ * the device-wide synchronisation of cudaMalloc / cudaFree. (The paper and its
+ * pages have no counterpart: this is a deployment variant of ckl_forward.)
+ * No handle is involved, since ckl_create allocates. The forward workspace and
+ * the device status word live in one file-scope device array of 32 MiB that
+ * every GPU which loads this library keeps until the process exits. A call whose
+ * T and chunk need more than that (32 MiB minus 256 bytes, as
+ * ckl_workspace_bytes would size the forward pass) is rejected with
+ * CKL_ERR_WORKSPACE before anything is enqueued. At V = 201088 and K = 100 a
+ * 4096-token chunk needs about 29 MiB plus 8 bytes per token of T.
+ * The first call on a device looks up the array's device address, the SM count
+ * and the TMA descriptor encoder for that device (with the device current); make
+ * that first call before any stream capture. Every call shares the array and
+ * clears the status word it needs; calls that overlap on the GPU (different
+ * streams or host threads) race on the array and must not be issued.
+ * Arguments are those of ckl_create (device, dtype, V, d, K) followed by those
+ * of ckl_forward without the workspace; chunk has no max_chunk bound other than
+ * the scratch size. loss_host: as in ckl_forward (pageable memory is fine). */
+ckl_status ckl_forward_static(int device, ckl_dtype dtype, int64_t V, int64_t d, int64_t K,
+                              const void* H, const void* W, const int32_t* topk_idx,
+                              const float* topk_logit, const uint8_t* mask, int64_t T,
+                              int64_t chunk, float* loss, float* token_lse, float* token_loss,
+                              void* stream, float* loss_host);
+
 /* Wait for `stream` and return the device-detected status of the calls enqueued
  * on it since the last synchronising call (clears it). */
 ckl_status ckl_sync_status(ckl_handle h, void* stream);
