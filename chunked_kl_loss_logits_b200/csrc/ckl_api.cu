@@ -98,13 +98,16 @@ struct WsPlan {
          off_Pk = 0, off_part = 0, off_G = 0, off_dHp = 0, total = 0;
 };
 
+// dH tiles are 256 x 256 outputs computed by CTA pairs; split the vocabulary
+// (the contraction) so that the tile count fills the pairs evenly.
 int pick_dh_split(int64_t Tc, int64_t d, int64_t V, int num_sms) {
-  const int64_t tiles = ((Tc + 127) / 128) * ((d + 191) / 192);
+  const int64_t tiles = ((Tc + 255) / 256) * ((d + 255) / 256);
   const int64_t n_kb = (V + 63) / 64;
+  const int units = std::max(1, num_sms / 2);
   int best = 1;
   double best_cost = 1e300;
   for (int s = 1; s <= 8 && s <= n_kb; ++s) {
-    const double waves = std::ceil((double)(tiles * s) / std::max(1, num_sms));
+    const double waves = std::ceil((double)(tiles * s) / units);
     const double cost = waves / s + 0.01 * s;  // time per unit of tile work, plus partial traffic
     if (cost < best_cost - 1e-9) { best_cost = cost; best = s; }
   }
@@ -253,7 +256,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     TcMaps mz;
     if (bf16) {
       if (!make_map(h, &mz.a, Hc, d, Tc, (uint64_t)d * 2, 64, 128) ||
-          !make_map(h, &mz.b, W, d, V, (uint64_t)d * 2, 64, 256))
+          !make_map(h, &mz.b, W, d, V, (uint64_t)d * 2, 64, 128))
         return CKL_ERR_CUDA;
       if (backward && !make_map(h, &mz.c, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 32))
         return CKL_ERR_CUDA;

@@ -362,12 +362,10 @@ void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* 
   const int h_bytes = (d * (int)sizeof(Tin) + 15) & ~15;
   const int k_bytes = (K * 4 + 15) & ~15;
   const size_t smem = (size_t)kGatherWarps * (h_bytes + 2 * k_bytes);
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The attribute is per device: set it whenever the launch needs more than the default.
+  if (smem > 48 * 1024)
     cudaFuncSetAttribute(gather_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         200 * 1024);
-    attr_set = true;
-  }
+                         (int)smem);
   gather_kernel<Tin><<<blocks_for(Tc, kGatherWarps), kGatherWarps * 32, smem, s>>>(
       H, W, idx, logit, t0, Tc, d, V, K, h_bytes, k_bytes, b.tok, b.zk, b.Pk, status);
 }

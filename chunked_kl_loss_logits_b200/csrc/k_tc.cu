@@ -15,19 +15,28 @@
 //   DW  : dW (+)= G^T H_c, contraction over the chunk's tokens; the epilogue adds
 //         its fp32 tile into dW with a TMA reduce-add (the add happens in L2).
 //
-// CTA layout (192 threads, one CTA per SM):
-//   warp 0      TMA producer: 128B-swizzled tiles of A and B into a STAGES-deep
-//               shared-memory ring (mbarrier full/empty pairs).
-//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
-//               (M=128, N=BN, K=16) into one of two TMEM accumulators and
-//               commits each stage back to the producer.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (thread = output row),
-//               the kind's math, then either plain stores or 128B-swizzled
-//               shared-memory staging + TMA bulk stores, overlapped with the MMA
-//               of the next tile through the second accumulator.
+// Work unit: a 256 x 256 output tile computed by a CTA pair (a cluster of two
+// CTAs on neighbouring SMs) with tcgen05.mma.cta_group::2: each CTA stages its
+// own 128 rows of A and its own 128 rows (K-major) or columns (MN-major) of B,
+// so a stage is 32 KB per CTA and the rings hold 6-7 stages. The pair's
+// accumulator is split by rows: rows 0-127 in the even CTA's TMEM, 128-255 in the
+// odd CTA's.
+//
+// CTA layout (192 threads, one CTA per SM, two CTAs per cluster):
+//   warp 0      TMA producer (both CTAs): tiles into the CTA's own ring; the
+//               copies signal the even CTA's `full` barrier, where the even
+//               producer has posted the byte count of both halves.
+//   warp 1      allocates 512 TMEM columns in both CTAs; in the even CTA one
+//               thread issues the pair MMAs (M=256, N=256, K=16) into one of two
+//               accumulators and commits each stage to the `empty` barriers of
+//               both CTAs (tcgen05.commit multicast).
+//   warps 2..5  epilogue (both CTAs): tcgen05.ld of the CTA's 128 accumulator
+//               rows (thread = row), the kind's math, plain stores or 128B-swizzled
+//               staging + TMA bulk stores, then one arrival per warp on the even
+//               CTA's `tempty` barrier.
 // Operand layouts: H, W and G are read K-major for LSE/GRAD/DH-A; W (DH-B), G
 // (DW-A) and H (DW-B) are read MN-major, so no operand is ever transposed in
-// memory. Every wait is bounded (common.cuh).
+// memory. No load uses cluster multicast. Every wait is bounded (common.cuh).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -35,7 +44,9 @@ namespace ckl {
 
 namespace {
 
-constexpr int BM = 128;
+constexpr int BM = 128;               // rows of A per CTA (256 per pair)
+constexpr int BN = 256;               // output columns per pair tile
+constexpr int BNH = BN / 2;           // rows/columns of B staged per CTA
 constexpr int BK = 64;                // 64 bf16 = one 128-byte swizzle row
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
@@ -43,20 +54,20 @@ constexpr int kAccStride = 256;       // TMEM columns between the two accumulato
 constexpr int kAtomBytes = 64 * 128;  // one 64 (MN) x 64 (K) MN-major box
 constexpr int kStageBufBytes = 4096;  // one epilogue staging box: 32 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint16_t kPairMask = 0x3;
 
 template <TcKind KIND>
 struct Cfg;
-template <> struct Cfg<TcKind::LSE>  { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 4; static constexpr bool STAGED = true; };
-template <> struct Cfg<TcKind::GRAD> { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 4; static constexpr bool STAGED = true; };
-template <> struct Cfg<TcKind::DH>   { static constexpr int BN = 192; static constexpr bool A_MN = false, B_MN = true;  static constexpr int STAGES = 5; static constexpr bool STAGED = false; };
-template <> struct Cfg<TcKind::DW>   { static constexpr int BN = 192; static constexpr bool A_MN = true,  B_MN = true;  static constexpr int STAGES = 4; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::LSE>  { static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::GRAD> { static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::DH>   { static constexpr bool A_MN = false, B_MN = true;  static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
+template <> struct Cfg<TcKind::DW>   { static constexpr bool A_MN = true,  B_MN = true;  static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
 
 template <TcKind KIND>
 struct Layout {
-  static constexpr int BN = Cfg<KIND>::BN;
   static constexpr int STAGES = Cfg<KIND>::STAGES;
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = BNH * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   // two staging boxes per epilogue warp
@@ -74,10 +85,10 @@ __device__ __forceinline__ TileCoord tile_coord(const TcLaunch& p, int n_m, int 
                                                 int tile) {
   TileCoord c;
   c.split = 0;
-  if (p.kind == TcKind::DW) {  // neighbouring CTAs share the A (gradient) tile
+  if (p.kind == TcKind::DW) {  // neighbouring pairs share the A (gradient) tile
     c.nt = tile % n_n;
     c.mt = tile / n_n;
-  } else {  // neighbouring CTAs share the B tile (W rows / columns)
+  } else {  // neighbouring pairs share the B tile (W rows / columns)
     c.mt = tile % n_m;
     const int r = tile / n_m;
     c.nt = r % n_n;
@@ -118,7 +129,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmC, const TcLaunch p) {
   using L = Layout<KIND>;
-  constexpr int BN = L::BN;
   constexpr int STAGES = L::STAGES;
   constexpr bool A_MN = Cfg<KIND>::A_MN, B_MN = Cfg<KIND>::B_MN;
 
@@ -127,16 +137,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* epi_smem = smem + L::RING_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::RING_BYTES + L::EPI_BYTES);
-  uint64_t* full = bars;                 // [STAGES]
-  uint64_t* empty = bars + STAGES;       // [STAGES]
-  uint64_t* tfull = bars + 2 * STAGES;   // [2]
-  uint64_t* tempty = tfull + 2;          // [2]
-  uint64_t* done = tempty + 2;           // [1]
+  uint64_t* full = bars;                 // [STAGES] used in the even CTA
+  uint64_t* empty = bars + STAGES;       // [STAGES] both CTAs
+  uint64_t* tfull = bars + 2 * STAGES;   // [2] both CTAs
+  uint64_t* tempty = tfull + 2;          // [2] used in the even CTA
+  uint64_t* done = tempty + 2;           // [1] even CTA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_m = (p.M + BM - 1) / BM;
+  const uint32_t rank = cluster_ctarank();  // 0: leader (issues MMAs), 1: peer
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int n_m = (p.M + 2 * BM - 1) / (2 * BM);
   const int n_n = (p.N + BN - 1) / BN;
   const int n_split = (KIND == TcKind::DH) ? p.n_split : 1;
   const int kps = (p.n_kb + n_split - 1) / n_split;
@@ -149,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4 * 32);
+      mbar_init(&tempty[b], 2 * 4);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -160,9 +172,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmB);
     if (Cfg<KIND>::STAGED) tma_prefetch_desc(&tmC);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 1) tmem_alloc_pair(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -173,50 +186,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued = 0, issued_phase = 0;  // per-stage bits: loaded at least once / last parity
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+      for (int tile = pair; ok && tile < n_tiles; tile += n_pairs) {
         const TileCoord c = tile_coord(p, n_m, n_n, kps, tile);
+        const int a_row0 = c.mt * 2 * BM + (int)rank * BM;  // this CTA's rows of A
+        const int b_row0 = c.nt * BN + (int)rank * BNH;     // this CTA's rows/columns of B
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           unsigned char* sA = smem + stage * L::STAGE_BYTES;
           unsigned char* sB = sA + L::A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+          const uint32_t fbar = cluster_map(&full[stage], 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::STAGE_BYTES);
           if (!A_MN) {
-            tma_load_2d(sA, &tmA, &full[stage], kb * BK, c.mt * BM);
+            tma_load_2d_pair(sA, &tmA, fbar, kb * BK, a_row0);
           } else {
 #pragma unroll
             for (int a = 0; a < BM / 64; ++a)
-              tma_load_2d(sA + a * kAtomBytes, &tmA, &full[stage], c.mt * BM + a * 64, kb * BK);
+              tma_load_2d_pair(sA + a * kAtomBytes, &tmA, fbar, a_row0 + a * 64, kb * BK);
           }
           if (!B_MN) {
-            tma_load_2d(sB, &tmB, &full[stage], kb * BK, c.nt * BN);
+            tma_load_2d_pair(sB, &tmB, fbar, kb * BK, b_row0);
           } else {
 #pragma unroll
-            for (int a = 0; a < BN / 64; ++a)
-              tma_load_2d(sB + a * kAtomBytes, &tmB, &full[stage], c.nt * BN + a * 64, kb * BK);
+            for (int a = 0; a < BNH / 64; ++a)
+              tma_load_2d_pair(sB + a * kAtomBytes, &tmB, fbar, b_row0 + a * 64, kb * BK);
           }
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      // Let every copy this thread issued land before the CTA can exit.
+      // Wait until the pair's MMAs have consumed every stage this thread filled
+      // (so no copy is in flight when the CTA exits).
       for (int s = 0; s < STAGES; ++s) {
         if (!((issued >> s) & 1u)) continue;
         const long long t0 = clock64();
-        while (!mbar_try_wait(&full[s], (issued_phase >> s) & 1u)) {
+        while (!mbar_try_wait(&empty[s], (issued_phase >> s) & 1u)) {
           if (clock64() - t0 > kWaitCycles) { atomicOr(p.status, (unsigned)ST_TIMEOUT); break; }
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, A_MN, B_MN);
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(2 * BM, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
+      for (int tile = pair; ok && tile < n_tiles; tile += n_pairs, ++it) {
         const TileCoord c = tile_coord(p, n_m, n_n, kps, tile);
         const int buf = it & 1;
         const uint32_t use = (uint32_t)(it >> 1);
@@ -236,16 +253,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      : umma_desc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? umma_desc_sw128(b0 + kk * 2048, kAtomBytes, 1024)
                                      : umma_desc_sw128(b0 + kk * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);
+          umma_commit_pair_mc(&empty[stage], kPairMask);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tfull[buf]);
+        umma_commit_pair_mc(&tfull[buf], kPairMask);
       }
       // Every MMA issued above has completed once `done` flips.
-      umma_commit(done);
+      umma_commit_pair(done);
       const long long t0 = clock64();
       while (!mbar_try_wait(done, 0)) {
         if (clock64() - t0 > kWaitCycles) { atomicOr(p.status, (unsigned)ST_TIMEOUT); break; }
@@ -254,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;          // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;   // accumulator row owned by this thread
+    const int row = q * 32 + lane;   // accumulator row owned by this thread (within the CTA)
     unsigned char* stg = epi_smem + q * 2 * kStageBufBytes;  // this warp's two staging boxes
     int nstage = 0;                  // staging boxes this warp has filled so far
     // Fill staging box (nstage & 1) from this thread's row and hand it to TMA.
@@ -275,17 +292,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     int it = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+    for (int tile = pair; tile < n_tiles; tile += n_pairs, ++it) {
       const TileCoord c = tile_coord(p, n_m, n_n, kps, tile);
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       if (!mbar_wait(&tfull[buf], use & 1u, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kAccStride);
-      const int grow = c.mt * BM + row;  // output row (token for LSE/GRAD/DH, vocab id for DW)
+      const int crow0 = c.mt * 2 * BM + (int)rank * BM;  // first output row of this CTA
+      const int grow = crow0 + row;  // output row (token for LSE/GRAD/DH, vocab id for DW)
       const bool row_ok = grow < p.M;
       const int col0 = c.nt * BN;
-      const int row0 = c.mt * BM + q * 32;  // first row of this warp's staging boxes
+      const int row0 = crow0 + q * 32;  // first row of this warp's staging boxes
 
       if constexpr (KIND == TcKind::LSE) {
         // (max, sum exp2) over the tile's valid columns, in log2 units.
@@ -400,44 +418,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[buf]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_map(&tempty[buf], 0));
     }
     if (Cfg<KIND>::STAGED && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // neither CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
 template <TcKind KIND>
 cudaError_t launch_kind(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
   using L = Layout<KIND>;
-  const int n_m = (p.M + BM - 1) / BM;
-  const int n_n = (p.N + L::BN - 1) / L::BN;
+  const int n_m = (p.M + 2 * BM - 1) / (2 * BM);
+  const int n_n = (p.N + BN - 1) / BN;
   const int n_tiles = n_m * n_n * (KIND == TcKind::DH ? p.n_split : 1);
   if (n_tiles <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int grid = n_tiles < p.num_sms ? n_tiles : p.num_sms;
-  tc_kernel<KIND><<<grid, kThreads, L::SMEM_BYTES, s>>>(maps.a, maps.b, maps.c, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // As many pairs as can be resident at once (one CTA per SM), at most one per tile.
+  static int max_pairs = 0;
+  if (max_pairs == 0) {
+    cfg.gridDim = dim3(2 * p.num_sms, 1, 1);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, tc_kernel<KIND>, &cfg) != cudaSuccess ||
+        clusters < 1)
+      clusters = p.num_sms / 2;
+    max_pairs = clusters;
+  }
+  const int pairs = n_tiles < max_pairs ? n_tiles : max_pairs;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  return cudaLaunchKernelEx(&cfg, tc_kernel<KIND>, maps.a, maps.b, maps.c, p);
 }
 
 }  // namespace
 
-int tc_bn(TcKind k) {
-  switch (k) {
-    case TcKind::LSE: return Cfg<TcKind::LSE>::BN;
-    case TcKind::GRAD: return Cfg<TcKind::GRAD>::BN;
-    case TcKind::DH: return Cfg<TcKind::DH>::BN;
-    default: return Cfg<TcKind::DW>::BN;
-  }
-}
+int tc_bn(TcKind) { return BN; }
 
 cudaError_t launch_tc(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
   switch (p.kind) {
