@@ -104,6 +104,42 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_bf16_32k.md")
+KERNEL_SOURCES = ("chunked_kl_loss_logits_b200/csrc/k_tc.cu", "chunked_kl_loss_logits_b200/csrc/common.cuh",
+                  "chunked_kl_loss_logits_b200/csrc/k_small.cu", "chunked_kl_loss_logits_b200/csrc/kernels.h")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str, chunk: int):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None.
+
+    The summary records a hash of the kernel sources it was measured on; a
+    changed kernel (or another workload) gives None.
+    """
+    import re
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        text = f.read()
+    m = re.search(r"<!-- traffic (.*?) -->", text)
+    if not m:
+        return None
+    kv = dict(x.split("=", 1) for x in m.group(1).split())
+    if kv.get("source") != kernel_source_hash() or kv.get("workload") != workload or \
+            int(kv.get("chunk", -1)) != chunk:
+        return None
+    val = kv.get(kernel)
+    return float(val) if val is not None else None
+
+
 def bus_id_of(dev: int) -> str:
     import torch
     p = torch.cuda.get_device_properties(dev)
@@ -265,14 +301,16 @@ def run_ours(args, w, rank, world, local_rank):
     if top["flops"] > 0:
         achieved = top["flops"] / top["launches"] / (avg_ms / 1e3) / 1e12
         roof = {"kernel": top["name"], "bound": "tensor", "achieved": achieved, "peak": pk_sus,
-                "unit": "TFLOP/s", "frac": achieved / pk_sus, "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / pk_sus,
+                "traffic": recorded_traffic(top["name"], w.name, chunk),
                 "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
                 "flops_per_launch": top["flops"] / top["launches"], "avg_launch_ms": avg_ms}
     else:
         achieved = top["bytes"] / top["launches"] / (avg_ms / 1e3) / 1e9
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         roof = {"kernel": top["name"], "bound": "hbm", "achieved": achieved, "peak": hbm,
-                "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": recorded_traffic(top["name"], w.name, chunk),
                 "peak_source": f"{peak_src} hbm_gbs", "avg_launch_ms": avg_ms}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
