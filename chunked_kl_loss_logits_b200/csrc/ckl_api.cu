@@ -6,13 +6,15 @@
 // in less <6GB VRAM" (README, "Full Chunked KL"):
 //   mask_count                      N = sum(mask), 1/N
 //   per chunk c (Tc tokens):
-//     gather                        teacher p, merged P, sum P log P, z at the K ids, sum P z
-//     LSE contraction               per-vocabulary-tile (max, sum exp) of z = H_c W^T;
-//                                   stored-exp mode also keeps e = exp(z - tile max), bf16
+//     teacher                       p, merged P, sum P log P; ids sorted with their p (bf16)
+//                                   (fp32: also z at the K ids and sum p z by dot products)
+//     LSE contraction               per-vocabulary-tile (max, sum exp) of z = H_c W^T and
+//                                   sum p z over the ids in the tile (bf16); stored-exp
+//                                   mode also keeps e = exp(z - tile max) in bf16
 //     combine                       lse_t, l_t, gradient multipliers
 //     stored-exp mode:  scale_e     G = e * (mask/N) M exp(tile max - lse)       (in place)
 //     recompute mode:   GRAD        G = (mask/N) M exp(z - lse), z formed again
-//     fixup                         G at the K ids: subtract (mask/N) P
+//     fixup                         G at the K ids: subtract (mask/N) P, in place
 //     DH contraction (+ reduce)     dH_c = G W
 //     DW contraction                dW (+)= G^T H_c   (TMA reduce-add into dW)
 //   loss_finalize                   loss = sum mask l / N
@@ -48,7 +50,7 @@ enum KernelId {
   KID_MASK = 0, KID_GATHER, KID_LSE, KID_COMBINE, KID_GRAD, KID_SCALE, KID_FIXUP, KID_DH,
   KID_DH_REDUCE, KID_DW, KID_LOSS, KID_COUNT
 };
-const char* kKernelNames[KID_COUNT] = {"mask_count", "gather_topk", "lse_gemm", "lse_combine",
+const char* kKernelNames[KID_COUNT] = {"mask_count", "teacher_topk", "lse_gemm", "lse_combine",
                                        "grad_gemm", "scale_e", "topk_fixup", "dh_gemm",
                                        "dh_reduce", "dw_gemm", "loss_finalize"};
 
@@ -95,7 +97,8 @@ struct WsPlan {
   int64_t ldG = 0;
   int n_split = 1; // dH contraction splits (bf16)
   size_t off_ell = 0, off_lse = 0, off_misc = 0, off_tok = 0, off_cst = 0, off_zk = 0,
-         off_Pk = 0, off_part = 0, off_G = 0, off_dHp = 0, total = 0;
+         off_Pk = 0, off_part = 0, off_xpart = 0, off_sid = 0, off_sp = 0, off_G = 0, off_dHp = 0,
+         total = 0;
 };
 
 // dH tiles are 256 x 256 outputs computed by CTA pairs; split the vocabulary
@@ -130,9 +133,15 @@ WsPlan plan(const ckl_ctx* h, int64_t T, int64_t chunk, bool backward) {
   p.off_lse = take((size_t)std::max<int64_t>(T, 1) * 4);
   p.off_tok = take((size_t)p.Tc * 16);
   p.off_cst = take((size_t)p.Tc * 16);
-  p.off_zk = take((size_t)p.Tc * h->K * 4);
   p.off_Pk = take((size_t)p.Tc * h->K * 4);
   p.off_part = take((size_t)p.n_vt * p.Tc * 8);
+  if (bf16) {
+    p.off_xpart = take((size_t)p.n_vt * p.Tc * 4);
+    p.off_sid = take((size_t)p.Tc * h->K * 4);
+    p.off_sp = take((size_t)p.Tc * h->K * 4);
+  } else {
+    p.off_zk = take((size_t)p.Tc * h->K * 4);
+  }
   if (backward) {
     p.off_G = take((size_t)p.Tc * p.ldG * (bf16 ? 2 : 4));
     if (bf16) p.off_dHp = take((size_t)p.n_split * p.Tc * h->d * 4);
@@ -217,9 +226,12 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
   b.misc = reinterpret_cast<Misc*>(base + P.off_misc);
   b.tok = reinterpret_cast<float4*>(base + P.off_tok);
   b.cst = reinterpret_cast<float4*>(base + P.off_cst);
-  b.zk = reinterpret_cast<float*>(base + P.off_zk);
+  b.zk = h->dtype == CKL_BF16 ? nullptr : reinterpret_cast<float*>(base + P.off_zk);
   b.Pk = reinterpret_cast<float*>(base + P.off_Pk);
   b.part = reinterpret_cast<float2*>(base + P.off_part);
+  b.xpart = h->dtype == CKL_BF16 ? reinterpret_cast<float*>(base + P.off_xpart) : nullptr;
+  b.sid = h->dtype == CKL_BF16 ? reinterpret_cast<int32_t*>(base + P.off_sid) : nullptr;
+  b.sp = h->dtype == CKL_BF16 ? reinterpret_cast<float*>(base + P.off_sp) : nullptr;
   b.G = backward ? base + P.off_G : nullptr;
   b.dHp = (backward && h->dtype == CKL_BF16) ? reinterpret_cast<float*>(base + P.off_dHp) : nullptr;
   float* ell_all = reinterpret_cast<float*>(base + P.off_ell);
@@ -240,15 +252,16 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     const double zflops = 2.0 * Tc * (double)V * d;
     const unsigned char* Hc = static_cast<const unsigned char*>(H) + (size_t)t0 * d * esz;
 
-    chk(L(KID_GATHER, 2.0 * Tc * K * d, (double)Tc * (K * 8.0 + d * esz + K * d * esz), [&] {
-      if (bf16)
-        launch_gather<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(H),
-                                     static_cast<const __nv_bfloat16*>(W), idx, logit, t0, Tc, d,
-                                     V, K, b, h->d_status, s);
-      else
+    if (bf16) {
+      chk(L(KID_GATHER, 0, (double)Tc * K * 16.0, [&] {
+        launch_teacher(idx, logit, t0, Tc, V, K, b, h->d_status, s);
+      }));
+    } else {
+      chk(L(KID_GATHER, 2.0 * Tc * K * d, (double)Tc * (K * 8.0 + d * esz + K * d * esz), [&] {
         launch_gather<float>(static_cast<const float*>(H), static_cast<const float*>(W), idx,
                              logit, t0, Tc, d, V, K, b, h->d_status, s);
-    }));
+      }));
+    }
 
     // bf16: z = H_c W^T on the tensor cores. Stored-exp mode also writes
     // e = exp(z - tile max) into the gradient buffer (map c) for the backward.
@@ -267,6 +280,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
         TcLaunch p{};
         p.kind = TcKind::LSE; p.M = Tc; p.N = V; p.n_kb = (d + 63) / 64; p.n_split = 1; p.V = V;
         p.part = b.part; p.part_ld = Tc; p.store_e = store_e ? 1 : 0;
+        p.sid = b.sid; p.sp = b.sp; p.xpart = b.xpart; p.K = K;
         p.status = h->d_status; p.num_sms = h->num_sms;
         launch_tc(mz, p, s);
       } else {
@@ -298,8 +312,8 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
       }));
     }
     chk(L(KID_FIXUP, 0, (double)Tc * K * (12.0 + 2 * esz), [&] {
-      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, P.ldG, b, !store_e, s);
-      else launch_fixup<float>(idx, t0, Tc, K, V, P.ldG, b, true, s);
+      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, P.ldG, b, false, s);
+      else launch_fixup<float>(idx, t0, Tc, K, V, P.ldG, b, false, s);
     }));
 
     unsigned char* dHc = static_cast<unsigned char*>(dH) + (size_t)t0 * d * esz;

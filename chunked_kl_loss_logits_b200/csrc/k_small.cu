@@ -1,5 +1,7 @@
 // Memory-bound kernels of the fused top-K forward-KL loss: the sparse teacher
-// term (a warp per token gathers the student logits at the K cached ids), the
+// term (a warp per token: teacher softmax, merged probabilities, entropy, and
+// the ids sorted for the forward contraction; the fp32 path also gathers the
+// student logits at the K cached ids by dot products), the
 // merge of per-vocabulary-tile log-sum-exp partials, the top-K correction of the
 // gradient tile, the split-K reduction of dH, and the mask count / loss mean.
 //
@@ -48,6 +50,81 @@ __device__ __forceinline__ float dot16(const uint4& a, const uint4& b, const __n
 }
 
 constexpr int kGatherWarps = 4;
+constexpr int kTeacherWarps = 8;
+
+// One warp per token of the chunk (bf16 path):
+//  1. stage the token's K ids and logits (16-byte loads when K % 4 == 0)
+//  2. p = softmax(logits); M = sum p; P_k = total p of slot k's id (repeats add)
+//  3. ent = sum_k p_k log P_k
+//  4. the (id, p) pairs in ascending id order (ties in slot order), for the
+//     forward contraction's epilogue to pick z at the ids and form sum_k p_k z_k
+__global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ logit, int64_t t0, int Tc, int V,
+    int K, int k_bytes, float4* __restrict__ tok, float* __restrict__ Pk_out,
+    int32_t* __restrict__ sid_out, float* __restrict__ sp_out, unsigned* status) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kTeacherWarps + warp;
+  if (i >= Tc) return;
+  const int64_t t = t0 + i;
+  int* sId = reinterpret_cast<int*>(smem + (size_t)warp * 2 * k_bytes);
+  float* sP = reinterpret_cast<float*>(smem + (size_t)warp * 2 * k_bytes + k_bytes);
+
+  const int32_t* idr = idx + t * K;
+  const float* lgr = logit + t * K;
+  if ((K & 3) == 0) {
+    for (int k4 = lane; k4 < (K >> 2); k4 += 32) {
+      reinterpret_cast<int4*>(sId)[k4] = __ldg(reinterpret_cast<const int4*>(idr) + k4);
+      reinterpret_cast<float4*>(sP)[k4] = __ldg(reinterpret_cast<const float4*>(lgr) + k4);
+    }
+  } else {
+    for (int k = lane; k < K; k += 32) {
+      sId[k] = __ldg(idr + k);
+      sP[k] = __ldg(lgr + k);
+    }
+  }
+  __syncwarp();
+  float mx = -INFINITY;
+  for (int k = lane; k < K; k += 32) mx = fmaxf(mx, sP[k]);
+  mx = warp_max(mx);
+  const bool live = mx > -INFINITY;
+  float se = 0.f;
+  for (int k = lane; k < K; k += 32) se += live ? expf(sP[k] - mx) : 0.f;
+  se = warp_sum(se);
+  __syncwarp();
+  for (int k = lane; k < K; k += 32) {
+    sP[k] = (live && se > 0.f) ? expf(sP[k] - mx) / se : 0.f;
+    const int id = sId[k];
+    if (id < 0 || id >= V) atomicOr(status, (unsigned)ST_INDEX_RANGE);
+  }
+  __syncwarp();
+  float ent = 0.f, Msum = 0.f;
+  for (int k = lane; k < K; k += 32) {
+    const int id = sId[k];
+    const float p = sP[k];
+    float P = 0.f;
+    int rank = 0;
+    bool first = true;
+    for (int j = 0; j < K; ++j) {
+      const int o = sId[j];
+      if (o == id) {
+        P += sP[j];
+        first = first && (j >= k);
+        rank += j < k;
+      } else {
+        rank += o < id;
+      }
+    }
+    if (p > 0.f) ent += p * logf(P);
+    Msum += p;
+    Pk_out[(int64_t)i * K + k] = first ? P : 0.f;
+    sid_out[(int64_t)i * K + rank] = id;
+    sp_out[(int64_t)i * K + rank] = p;
+  }
+  ent = warp_sum(ent);
+  Msum = warp_sum(Msum);
+  if (lane == 0) tok[i] = make_float4(ent, 0.f, Msum, 0.f);
+}
 
 // One warp per token of the chunk.
 //  1. stage the token's K ids and logits (16-byte loads when K % 4 == 0) and H row
@@ -188,12 +265,13 @@ constexpr int kCombTok = 32, kCombSplit = 8;
 // reads of 32 consecutive tokens), then one warp merges the 8 results.
 __global__ void __launch_bounds__(kCombTok * kCombSplit) combine_kernel(
     int64_t t0, int Tc, int n_vt, const uint8_t* __restrict__ mask,
-    const float2* __restrict__ part, const float4* __restrict__ tok, const Misc* __restrict__ misc,
+    const float2* __restrict__ part, const float* __restrict__ xpart,
+    const float4* __restrict__ tok, const Misc* __restrict__ misc,
     float4* __restrict__ cst, float* __restrict__ lse_all, float* __restrict__ ell_all) {
-  __shared__ float sm[kCombSplit][kCombTok], ss[kCombSplit][kCombTok];
+  __shared__ float sm[kCombSplit][kCombTok], ss[kCombSplit][kCombTok], sx[kCombSplit][kCombTok];
   const int tk = threadIdx.x % kCombTok, sp = threadIdx.x / kCombTok;
   const int i = blockIdx.x * kCombTok + tk;
-  float m2 = -INFINITY, s = 0.f;
+  float m2 = -INFINITY, s = 0.f, x = 0.f;
   if (i < Tc) {
 #pragma unroll 4
     for (int j = sp; j < n_vt; j += kCombSplit) {
@@ -204,22 +282,27 @@ __global__ void __launch_bounds__(kCombTok * kCombSplit) combine_kernel(
       } else {
         s += q.y * ex2_approx(q.x - m2);
       }
+      if (xpart) x += xpart[(int64_t)j * Tc + i];
     }
   }
   sm[sp][tk] = m2;
   ss[sp][tk] = s;
+  sx[sp][tk] = x;
   __syncthreads();
   if (sp != 0 || i >= Tc) return;
   float M2 = -INFINITY;
 #pragma unroll
   for (int j = 0; j < kCombSplit; ++j) M2 = fmaxf(M2, sm[j][tk]);
-  float S = 0.f;
+  float S = 0.f, X = 0.f;
 #pragma unroll
-  for (int j = 0; j < kCombSplit; ++j)
+  for (int j = 0; j < kCombSplit; ++j) {
     if (sm[j][tk] > -INFINITY) S += ss[j][tk] * ex2_approx(sm[j][tk] - M2);
+    X += sx[j][tk];
+  }
   const float lse = (M2 + log2f(S)) * kLn2;
   const float4 t4 = tok[i];
-  const float ell = t4.x - t4.y + t4.z * lse;
+  const float cross = xpart ? X : t4.y;  // bf16: from the contraction's epilogue; fp32: gathered
+  const float ell = t4.x - cross + t4.z * lse;
   const int64_t t = t0 + i;
   const float sc = (mask == nullptr || mask[t] != 0) ? misc->invN : 0.f;
   cst[i] = make_float4(lse, sc * t4.z, sc, 0.f);
@@ -355,6 +438,16 @@ void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t 
   mask_count_kernel<<<1, kReduceThreads, 0, s>>>(mask, T, misc);
 }
 
+void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V, int K,
+                    const ChunkBufs& b, unsigned* status, cudaStream_t s) {
+  const int k_bytes = (K * 4 + 15) & ~15;
+  const size_t smem = (size_t)kTeacherWarps * 2 * k_bytes;
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(teacher_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  teacher_kernel<<<blocks_for(Tc, kTeacherWarps), kTeacherWarps * 32, smem, s>>>(
+      idx, logit, t0, Tc, V, K, k_bytes, b.tok, b.Pk, b.sid, b.sp, status);
+}
+
 template <typename Tin>
 void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* logit, int64_t t0,
                    int Tc, int d, int V, int K, const ChunkBufs& b, unsigned* status,
@@ -372,14 +465,11 @@ void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* 
 template void launch_gather<float>(const float*, const float*, const int32_t*, const float*,
                                    int64_t, int, int, int, int, const ChunkBufs&, unsigned*,
                                    cudaStream_t);
-template void launch_gather<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
-                                           const int32_t*, const float*, int64_t, int, int, int,
-                                           int, const ChunkBufs&, unsigned*, cudaStream_t);
 
 void launch_combine(int64_t t0, int Tc, int n_vt, const uint8_t* mask, const ChunkBufs& b,
                     float* lse_all, float* ell_all, cudaStream_t s) {
   combine_kernel<<<blocks_for(Tc, kCombTok), kCombTok * kCombSplit, 0, s>>>(
-      t0, Tc, n_vt, mask, b.part, b.tok, b.misc, b.cst, lse_all, ell_all);
+      t0, Tc, n_vt, mask, b.part, b.xpart, b.tok, b.misc, b.cst, lse_all, ell_all);
 }
 
 void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s) {

@@ -6,7 +6,8 @@
 // normaliser is being accumulated, and the backward pass needs the analytic
 // gradient of each chunk):
 //   LSE : z = H_c W^T tile by tile; the epilogue keeps each row's (max, sum of
-//         exp) over the tile's vocabulary columns. With `store_e` it also writes
+//         exp) over the tile's vocabulary columns, and sum_k p_k z_k over the
+//         row's cached teacher ids that fall in the tile. With `store_e` it also writes
 //         e = exp(z - tile max) in bf16 to the chunk's gradient buffer, so the
 //         backward pass can rescale it instead of forming z again.
 //   GRAD: z formed again; the epilogue writes G = gmul * exp(z - lse) in bf16.
@@ -15,10 +16,11 @@
 //   DW  : dW (+)= G^T H_c, contraction over the chunk's tokens; the epilogue adds
 //         its fp32 tile into dW with a TMA reduce-add (the add happens in L2).
 //
-// Work unit: a 256 x 256 output tile computed by a CTA pair (a cluster of two
+// Work unit: a 256 x BN output tile computed by a CTA pair (a cluster of two
 // CTAs on neighbouring SMs) with tcgen05.mma.cta_group::2: each CTA stages its
-// own 128 rows of A and its own 128 rows (K-major) or columns (MN-major) of B,
-// so a stage is 32 KB per CTA and the rings hold 6-7 stages. The pair's
+// own 128 rows of A and its own BN/2 rows (K-major) or columns (MN-major) of B,
+// so a stage is 32 KB per CTA and the rings hold 6-7 stages (BN = 256; a 192-wide
+// dW tile with a transposed copy of H measured slower, 39 vs 34 ms per step). The pair's
 // accumulator is split by rows: rows 0-127 in the even CTA's TMEM, 128-255 in the
 // odd CTA's.
 //
@@ -45,8 +47,6 @@ namespace ckl {
 namespace {
 
 constexpr int BM = 128;               // rows of A per CTA (256 per pair)
-constexpr int BN = 256;               // output columns per pair tile
-constexpr int BNH = BN / 2;           // rows/columns of B staged per CTA
 constexpr int BK = 64;                // 64 bf16 = one 128-byte swizzle row
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
@@ -58,16 +58,20 @@ constexpr uint16_t kPairMask = 0x3;
 
 template <TcKind KIND>
 struct Cfg;
-template <> struct Cfg<TcKind::LSE>  { static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
-template <> struct Cfg<TcKind::GRAD> { static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
-template <> struct Cfg<TcKind::DH>   { static constexpr bool A_MN = false, B_MN = true;  static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
-template <> struct Cfg<TcKind::DW>   { static constexpr bool A_MN = true,  B_MN = true;  static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
+// BN: output columns per pair tile (each CTA stages BN/2 rows or columns of B).
+template <> struct Cfg<TcKind::LSE>  { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::GRAD> { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::DH>   { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = true;  static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
+template <> struct Cfg<TcKind::DW>   { static constexpr int BN = 256; static constexpr bool A_MN = true,  B_MN = true;  static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
 
 template <TcKind KIND>
 struct Layout {
+  static constexpr int BN = Cfg<KIND>::BN;
+  static constexpr int BNH = BN / 2;
   static constexpr int STAGES = Cfg<KIND>::STAGES;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BNH * BK * 2;
+  static_assert(!Cfg<KIND>::B_MN || BNH % 64 == 0, "MN-major B is staged in 64-column atoms");
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   // two staging boxes per epilogue warp
@@ -108,6 +112,14 @@ __device__ __forceinline__ void stage_row(unsigned char* box, int r, const uint4
   for (int c = 0; c < 8; ++c) rowp[c ^ (r & 7)] = chunks[c];
 }
 
+// v[i] for a runtime index 0 <= i < 32, by selects (the array stays in registers).
+__device__ __forceinline__ float pick32(const float (&v)[32], int i) {
+  float r = v[0];
+#pragma unroll
+  for (int t = 1; t < 32; ++t) r = (i == t) ? v[t] : r;
+  return r;
+}
+
 // Pack 32 + 32 fp32 values as 64 bf16 (one staged row of a 64-column box).
 __device__ __forceinline__ void pack_row_bf16(const float (&a)[32], const float (&b)[32],
                                               uint4 (&out)[8]) {
@@ -130,6 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const __grid_constant__ CUtensorMap tmC, const TcLaunch p) {
   using L = Layout<KIND>;
   constexpr int STAGES = L::STAGES;
+  constexpr int BN = L::BN, BNH = L::BNH;
   constexpr bool A_MN = Cfg<KIND>::A_MN, B_MN = Cfg<KIND>::B_MN;
 
   extern __shared__ unsigned char smem_raw[];
@@ -306,17 +319,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = crow0 + q * 32;  // first row of this warp's staging boxes
 
       if constexpr (KIND == TcKind::LSE) {
-        // (max, sum exp2) over the tile's valid columns, in log2 units.
+        // (max, sum exp2) over the tile's valid columns, in log2 units; on the same
+        // pass, sum p_k z_k over the row's cached ids that fall in this tile (the
+        // ids are sorted, so a cursor advances with the columns).
+        const int32_t* srow = p.sid + (int64_t)grow * p.K;
+        const float* prow = p.sp + (int64_t)grow * p.K;
+        int j = p.K;
+        if (row_ok) {
+          int lo = 0, hi = p.K;  // first sorted id >= col0
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(srow + mid) < col0) lo = mid + 1; else hi = mid;
+          }
+          j = lo;
+        }
+        int nid = j < p.K ? __ldg(srow + j) : INT_MAX;
+        float cross = 0.f;
         float m2 = -INFINITY;
 #pragma unroll 1
         for (int cc = 0; cc < BN / 32; ++cc) {
           float v[32];
           tmem_ld32(taddr + cc * 32, v);
           const int cb = col0 + cc * 32;
+          while (nid < cb + 32) {
+            if (nid < p.V) cross += __ldg(prow + j) * pick32(v, nid - cb);
+            ++j;
+            nid = j < p.K ? __ldg(srow + j) : INT_MAX;
+          }
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (cb + j < p.V) m2 = fmaxf(m2, v[j] * kLog2e);
+          for (int jj = 0; jj < 32; ++jj)
+            if (cb + jj < p.V) m2 = fmaxf(m2, v[jj] * kLog2e);
         }
+        if (row_ok) p.xpart[(int64_t)c.nt * p.part_ld + grow] = cross;
         float s = 0.f;
         if (!p.store_e) {
 #pragma unroll 1
@@ -437,7 +471,7 @@ template <TcKind KIND>
 cudaError_t launch_kind(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
   using L = Layout<KIND>;
   const int n_m = (p.M + 2 * BM - 1) / (2 * BM);
-  const int n_n = (p.N + BN - 1) / BN;
+  const int n_n = (p.N + L::BN - 1) / L::BN;
   const int n_tiles = n_m * n_n * (KIND == TcKind::DH ? p.n_split : 1);
   if (n_tiles <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -471,7 +505,14 @@ cudaError_t launch_kind(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
 
 }  // namespace
 
-int tc_bn(TcKind) { return BN; }
+int tc_bn(TcKind k) {
+  switch (k) {
+    case TcKind::LSE: return Cfg<TcKind::LSE>::BN;
+    case TcKind::GRAD: return Cfg<TcKind::GRAD>::BN;
+    case TcKind::DH: return Cfg<TcKind::DH>::BN;
+    default: return Cfg<TcKind::DW>::BN;
+  }
+}
 
 cudaError_t launch_tc(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
   switch (p.kind) {

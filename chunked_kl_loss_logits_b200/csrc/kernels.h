@@ -18,6 +18,9 @@ struct ChunkBufs {
   float* Pk;     // Tc x K total teacher probability of each slot's id; 0 on every slot
                  // but the first that holds a given id (so each id is corrected once)
   float2* part;  // n_vt x Tc partial (max, sum) of exp over one vocabulary tile, log2 units
+  float* xpart;  // bf16: n_vt x Tc partial sum_k p_k z_k over the ids inside one vocabulary tile
+  int32_t* sid;  // bf16: Tc x K cached ids of each token, ascending
+  float* sp;     // bf16: Tc x K teacher probability of each sorted slot
   void* G;       // Tc x ldG scaled gradient of the logits (bf16 or f32)
   float* dHp;    // split-K partials of dH (bf16 path)
   struct Misc* misc;
@@ -33,6 +36,11 @@ struct Misc {
 
 // ---- small kernels (k_small.cu)
 void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t s);
+// bf16: teacher softmax, merged P, entropy term and each token's ids sorted with
+// their probabilities (the forward contraction picks the student logits there).
+void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V, int K,
+                    const ChunkBufs& b, unsigned* status, cudaStream_t s);
+// fp32: as launch_teacher, plus the student logits at the ids by dot products.
 template <typename Tin>
 void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* logit, int64_t t0,
                    int Tc, int d, int V, int K, const ChunkBufs& b, unsigned* status,
@@ -74,6 +82,10 @@ struct TcLaunch {
   int V;           // LSE / GRAD: number of valid vocabulary columns
   float2* part;    // LSE
   int part_ld;     // LSE: rows of one vocabulary tile's partials (= Tc)
+  const int32_t* sid;  // LSE: sorted cached ids per row (Tc x K)
+  const float* sp;     // LSE: their teacher probabilities
+  float* xpart;        // LSE: per-tile partial cross term, same layout as part
+  int K;
   int store_e;     // LSE: also store exp(z - tile max) in bf16 through map c
   const float4* cst;  // GRAD
   uint16_t* G;        // GRAD

@@ -132,7 +132,7 @@ ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t
  * T and chunk need more than that (32 MiB minus 256 bytes, as
  * ckl_workspace_bytes would size the forward pass) is rejected with
  * CKL_ERR_WORKSPACE before anything is enqueued. At V = 201088 and K = 100 a
- * 4096-token chunk needs about 29 MiB plus 8 bytes per token of T.
+ * 2048-token chunk needs about 21 MiB plus 8 bytes per token of T.
  * The first call on a device looks up the array's device address, the SM count
  * and the TMA descriptor encoder for that device (with the device current); make
  * that first call before any stream capture. Every call shares the array and

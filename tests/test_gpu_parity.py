@@ -231,8 +231,8 @@ def test_launch_count_and_profiling():
     h.fwd_bwd(H, W, idx, logit, mask, chunk=128)
     stats = {s["name"]: s for s in h.profile_collect()}
     n1 = h.launch_count()
-    # mask count + 2 chunks x (gather, lse, combine, scale_e, fixup, dh, dh_reduce, dw) + loss
+    # mask count + 2 chunks x (teacher, lse, combine, scale_e, fixup, dh, dh_reduce, dw) + loss
     assert n1 - n0 == 1 + 2 * 8 + 1
-    for k in ("lse_gemm", "scale_e", "dh_gemm", "dw_gemm", "gather_topk"):
+    for k in ("lse_gemm", "scale_e", "dh_gemm", "dw_gemm", "teacher_topk"):
         assert stats[k]["launches"] == 2 and stats[k]["total_ms"] > 0
     assert stats["lse_gemm"]["flops"] == pytest.approx(2 * 256 * 1000 * 64)
