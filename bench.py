@@ -140,6 +140,22 @@ def recorded_traffic(kernel: str, workload: str, chunk: int):
     return float(val) if val is not None else None
 
 
+def max_over_ranks(ms: float, world: int, device="cpu") -> float:
+    """The slowest rank's time: every rank takes part, every rank gets the max."""
+    if world == 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, steps: int, ms_max: float) -> float:
+    """Weak scaling: every rank processes its own batch; the job rate uses the slowest rank."""
+    return tokens_per_rank * world * steps / (ms_max / 1e3)
+
+
 def bus_id_of(dev: int) -> str:
     import torch
     p = torch.cuda.get_device_properties(dev)
@@ -245,11 +261,7 @@ def run_ours(args, w, rank, world, local_rank):
     clocks = sampler.stop()
     launches = h.launch_count() - n_launch0
     h.sync_status()
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(e0.elapsed_time(e1), world, dev)
     stats = h.profile_collect()
     h.profile_enable(False, 0)
     peak_mem = torch.cuda.max_memory_allocated(dev) / 2**30
@@ -272,10 +284,7 @@ def run_ours(args, w, rank, world, local_rank):
     f1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    t2 = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t2.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -287,8 +296,7 @@ def run_ours(args, w, rank, world, local_rank):
         return
 
     peaks, peak_src = load_peaks()
-    tokens = w.T * world * args.steps
-    value = tokens / (ms_max / 1e3)
+    value = job_tokens_per_s(w.T, world, args.steps, ms_max)
     step_ms = ms_max / args.steps
     useful = 6.0 * w.T * w.V * w.d
     executed = 8.0 * w.T * w.V * w.d
@@ -329,7 +337,7 @@ def run_ours(args, w, rank, world, local_rank):
         "peak_mem_gib": peak_mem,
         "roofline": roof,
         "cpu_baseline": cpu,
-        "e2e": {"value": w.T * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(w.T, world, args.steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
         "gpu_launches": launches,
         "clocks": clocks,
