@@ -221,13 +221,15 @@ def run_ours(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     chunk = args.chunk or w.chunk
     x = make_inputs(w, seed=w.seed + 7919 * rank)
-    H = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
-    W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    H = torch.from_numpy(x["H"]).to(dev).to(tdt)
+    W = torch.from_numpy(x["W"]).to(dev).to(tdt)
     idx = torch.from_numpy(x["idx"]).to(dev)
     logit = torch.from_numpy(x["logit"]).to(dev)
     mask = None if x["mask"] is None else torch.from_numpy(x["mask"]).to(dev)
-    h = ckl.ChunkedKL(w.V, w.d, w.K, dtype=torch.bfloat16, max_chunk=chunk, device=dev)
-    h.set_recompute(args.recompute)
+    h = ckl.ChunkedKL(w.V, w.d, w.K, dtype=tdt, max_chunk=chunk, device=dev)
+    if w.dtype == "bf16":
+        h.set_recompute(args.recompute)
     ws = h.workspace(w.T, chunk)
     out = (torch.empty((), dtype=torch.float32, device=dev), torch.empty_like(H),
            torch.empty((w.V, w.d), dtype=torch.float32, device=dev))
@@ -273,7 +275,8 @@ def run_ours(args, w, rank, world, local_rank):
     mh = None if mask is None else mask.cpu().pin_memory()
     stag = (torch.empty_like(H), torch.empty_like(idx), torch.empty_like(logit),
             None if mask is None else torch.empty_like(mask))
-    h2d = Hh.numel() * 2 + ih.numel() * 4 + lh.numel() * 4 + (0 if mh is None else mh.numel())
+    h2d = Hh.numel() * Hh.element_size() + ih.numel() * 4 + lh.numel() * 4 + \
+        (0 if mh is None else mh.numel())
     h.fwd_bwd_from_host(Hh, ih, lh, mh, stag, W, chunk, out, ws)
     barrier()
     torch.cuda.synchronize(dev)
@@ -299,7 +302,8 @@ def run_ours(args, w, rank, world, local_rank):
     value = job_tokens_per_s(w.T, world, args.steps, ms_max)
     step_ms = ms_max / args.steps
     useful = 6.0 * w.T * w.V * w.d
-    executed = 8.0 * w.T * w.V * w.d
+    recompute = args.recompute or w.dtype != "bf16"
+    executed = (8.0 if recompute else 6.0) * w.T * w.V * w.d  # stored mode forms the logits once
     pk_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     pk_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     kern = sorted(stats, key=lambda s: -s["total_ms"])
@@ -323,10 +327,12 @@ def run_ours(args, w, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
         "config": {"workload": w.name, "T": w.T, "d": w.d, "V": w.V, "K": w.K, "chunk": chunk,
-                   "backward": "recompute logits" if args.recompute else "stored exp(z), bf16",
+                   "backward": ("recompute logits" if args.recompute or w.dtype != "bf16"
+                                else "stored exp(z), bf16"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "no flush: inputs larger than L2 (W alone is 1.16 GB)"},
         "tflops_useful": useful / (step_ms / 1e3) / 1e12,
@@ -352,6 +358,74 @@ def run_ours(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args, w):
+    """256K-token workload: throughput vs chunk, and peak device memory vs T.
+
+    Prints one JSON line per point (kind "chunk_sweep" or "memory_sweep"). Peak
+    memory counts everything the step allocates through torch: inputs, outputs
+    and the library's workspace.
+    """
+    import torch
+
+    from chunked_kl_loss_logits_b200 import ckl
+    from chunked_kl_loss_logits_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS["bf16_256k"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    x = make_inputs(w)
+    H_all = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
+    W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+    idx_all = torch.from_numpy(x["idx"]).to(dev)
+    lg_all = torch.from_numpy(x["logit"]).to(dev)
+    del x
+    stream = torch.cuda.current_stream(dev)
+    for chunk in w.chunk_sweep:
+        h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=chunk, device=dev)
+        ws = h.workspace(w.T, chunk)
+        out = (torch.empty((), device=dev), torch.empty_like(H_all),
+               torch.empty((w.V, w.d), dtype=torch.float32, device=dev))
+        for _ in range(2):
+            h.fwd_bwd(H_all, W, idx_all, lg_all, None, chunk=chunk, out=out, workspace=ws, sync=False)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_chunks = (w.T + chunk - 1) // chunk
+        h.profile_enable(True, args.sweep_steps * (10 * n_chunks + 8))
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.sweep_steps):
+            h.fwd_bwd(H_all, W, idx_all, lg_all, None, chunk=chunk, out=out, workspace=ws, sync=False)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        h.sync_status()
+        ms = e0.elapsed_time(e1) / args.sweep_steps
+        kern = {k["name"]: round(k["total_ms"] / args.sweep_steps, 2) for k in h.profile_collect()}
+        print(json.dumps({"kind": "chunk_sweep", "workload": w.name, "T": w.T, "chunk": chunk,
+                          "ms_per_step": ms, "tokens_per_s": w.T / (ms / 1e3),
+                          "tflops_useful": 6.0 * w.T * w.V * w.d / (ms / 1e3) / 1e12,
+                          "workspace_gib": ws.numel() / 2**30, "kernel_ms_per_step": kern}),
+              flush=True)
+        del out, ws
+        h.close()
+    chunk = 4096
+    for T in (4096, 8192, 16384, 32768, 65536, 131072, 262144):
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+        H = H_all[:T].clone()
+        idx = idx_all[:T].clone()
+        lg = lg_all[:T].clone()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=chunk, device=dev)
+        loss, dH, dW = h.fwd_bwd(H, W, idx, lg, None, chunk=chunk)
+        torch.cuda.synchronize(dev)
+        peak = torch.cuda.max_memory_allocated(dev)
+        print(json.dumps({"kind": "memory_sweep", "workload": w.name, "T": T, "chunk": chunk,
+                          "peak_gib_step": (peak - base) / 2**30,
+                          "peak_gib_with_inputs": (peak - base + (H.numel() * 2 + idx.numel() * 8)) / 2**30,
+                          "resident_W_gib": W.numel() * 2 / 2**30}), flush=True)
+        del loss, dH, dW, H, idx, lg
+        h.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -361,6 +435,9 @@ def main():
     ap.add_argument("--workload", default="bf16_32k")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="256K workload: throughput vs chunk and peak memory vs T (extra JSON lines)")
+    ap.add_argument("--sweep-steps", type=int, default=3)
     ap.add_argument("--recompute", action="store_true",
                     help="form the logits again in the backward instead of keeping exp(z)")
     args = ap.parse_args()
@@ -377,6 +454,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, w, rank, world)
+        return
+    if args.sweep:
+        run_sweep(args, w)
         return
     if world > 1:
         import datetime

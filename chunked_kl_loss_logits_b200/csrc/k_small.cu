@@ -257,12 +257,12 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
   if (lane == 0) tok[i] = make_float4(ent, cross, Msum, 0.f);
 }
 
-constexpr int kCombTok = 32, kCombSplit = 8;
+constexpr int kCombTok = 32, kCombSplit = 32;
 
 // Merge the per-vocabulary-tile (max, sum) partials into logsumexp(z_t), then
 // l_t = ent - cross + M lse and the gradient multipliers. A block covers 32
-// tokens; its 8 warps each merge every 8th vocabulary tile (coalesced 256-byte
-// reads of 32 consecutive tokens), then one warp merges the 8 results.
+// tokens; its 32 warps each merge every 32nd vocabulary tile (coalesced 256-byte
+// reads of 32 consecutive tokens), then one warp merges the 32 results.
 __global__ void __launch_bounds__(kCombTok * kCombSplit) combine_kernel(
     int64_t t0, int Tc, int n_vt, const uint8_t* __restrict__ mask,
     const float2* __restrict__ part, const float* __restrict__ xpart,
