@@ -164,3 +164,21 @@ def sampled_rows(H, W, idx, logit, rows, mask=None, with_dW=False):
     if with_dW:
         out["dW_part"] = Gs.T @ np.asarray(Hr, dtype=F64)
     return out
+
+
+def topk_cache(H, W, K):
+    """Teacher top-K cache: per token, the K largest logits of z = H W^T and their ids.
+
+    The offline distillation of "Efficient Knowledge Distillation for LLMs:
+    Offline Top-K Logits and a Fused Chunked KL Loss" (abstract) and the author's
+    forum post: the teacher's forward pass runs once and each position keeps only
+    its largest logits (100 of them), which the loss above then reads. Order:
+    descending logit; equal logits in ascending id order. Returns (idx int64
+    (T, K), logit float64 (T, K)). Computed in float64 from the exact inputs.
+    """
+    z = student_logits(H, W)
+    T, V = z.shape
+    K = min(K, V)
+    ids = np.broadcast_to(np.arange(V), z.shape)
+    order = np.lexsort((ids, -z), axis=1)[:, :K]   # primary key -z, then id
+    return order.astype(np.int64), np.take_along_axis(z, order, axis=1)
