@@ -21,6 +21,7 @@ Prints one JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -426,6 +427,55 @@ def run_sweep(args, w):
         h.close()
 
 
+def run_topk_cache(args, w):
+    """Teacher top-K cache builder on one workload's shape: tokens/s of one cache pass.
+
+    The teacher here has the student's shape (same V and d); its hidden states
+    are the workload's H. Prints one JSON line (kind "topk_cache"). The builder
+    forms every logit twice (a max pass and an emit pass), so it executes 4TVd
+    flops for the 2TVd of one logit contraction.
+    """
+    import torch
+
+    from chunked_kl_loss_logits_b200 import ckl
+    from chunked_kl_loss_logits_b200.workloads import make_inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    x = make_inputs(w)
+    H = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
+    W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+    del x
+    chunk = args.chunk or w.chunk
+    h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=chunk, device=dev)
+    n = ctypes.c_size_t()
+    ckl._check(ckl.lib().ckl_topk_workspace_bytes(h._h, w.T, chunk, ctypes.byref(n)), "ws")
+    ws = torch.empty(max(1, n.value), dtype=torch.uint8, device=dev)
+    for _ in range(max(1, args.warmup)):
+        h.topk_cache(H, W, chunk=chunk, workspace=ws, sync=False)
+    stream = torch.cuda.current_stream(dev)
+    n_chunks = (w.T + chunk - 1) // chunk
+    h.profile_enable(True, args.steps * 4 * n_chunks + 8)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        ids, lg = h.topk_cache(H, W, chunk=chunk, workspace=ws, sync=False)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    h.sync_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    kern = {k["name"]: round(k["total_ms"] / args.steps, 3) for k in h.profile_collect()}
+    peaks, src = load_peaks()
+    tf = 4.0 * w.T * w.V * w.d / (ms / 1e3) / 1e12
+    print(json.dumps({"kind": "topk_cache", "workload": w.name, "T": w.T, "V": w.V, "d": w.d,
+                      "K": w.K, "chunk": chunk, "steps": args.steps, "ms_per_pass": ms,
+                      "tokens_per_s": w.T / (ms / 1e3), "tflops_executed": tf,
+                      "frac_of_sustained_bf16": tf / peaks["bf16_tflops_sustained"], "peak_source": src,
+                      "workspace_mib": ws.numel() / 2**20, "kernel_ms_per_pass": kern}),
+          flush=True)
+    h.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -438,6 +488,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="256K workload: throughput vs chunk and peak memory vs T (extra JSON lines)")
     ap.add_argument("--sweep-steps", type=int, default=3)
+    ap.add_argument("--topk-cache", action="store_true",
+                    help="time the teacher top-K cache builder on the workload's shape instead")
     ap.add_argument("--recompute", action="store_true",
                     help="form the logits again in the backward instead of keeping exp(z)")
     args = ap.parse_args()
@@ -457,6 +509,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args, w)
+        return
+    if args.topk_cache:
+        run_topk_cache(args, w)
         return
     if world > 1:
         import datetime

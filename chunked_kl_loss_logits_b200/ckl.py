@@ -20,7 +20,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "ckl.h")
 F32, BF16 = 0, 1
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported size", 3: "workspace",
            4: "top-K index out of range", 5: "CUDA error", 6: "device wait timed out",
-           7: "pointer misaligned"}
+           7: "pointer misaligned", 8: "internal consistency check failed"}
 
 
 class CKLError(RuntimeError):
@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         "ckl_sync_status": ([_P, _P], ctypes.c_int),
         "ckl_launch_count": ([_P], ctypes.c_int64),
         "ckl_set_recompute": ([_P, ctypes.c_int], ctypes.c_int),
+        "ckl_topk_workspace_bytes": ([_P, _I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
+        "ckl_topk_cache": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _SZ, _P, ctypes.c_int], ctypes.c_int),
         "ckl_profile_enable": ([_P, ctypes.c_int, ctypes.c_int], ctypes.c_int),
         "ckl_profile_collect": ([_P, ctypes.POINTER(KernelStat), ctypes.c_int,
                                  ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -215,6 +217,30 @@ class ChunkedKL:
                                  ctypes.c_void_p(s.cuda_stream),
                                  ctypes.byref(host) if sync else None), "ckl_forward")
         return (loss, lse, ell) if token_stats else loss
+
+    def topk_cache(self, H, W, chunk: int | None = None, workspace=None, sync: bool = True,
+                   stream=None):
+        """Teacher top-K cache: (ids int32 T x K, logits float32 T x K), descending.
+
+        The handle must have the teacher's shape (V, d = teacher hidden size, K).
+        """
+        T = H.shape[0]
+        if H.dtype != self.dtype or W.dtype != self.dtype or H.shape[1] != self.d or \
+                tuple(W.shape) != (self.V, self.d):
+            raise ValueError("H must be T x d and W must be V x d, in the handle's dtype")
+        chunk = min(chunk or self.max_chunk, self.max_chunk)
+        idx = torch.empty((T, self.K), dtype=torch.int32, device=self.device)
+        logit = torch.empty((T, self.K), dtype=torch.float32, device=self.device)
+        if workspace is None:
+            n = _SZ()
+            _check(lib().ckl_topk_workspace_bytes(self._h, T, chunk, ctypes.byref(n)),
+                   "ckl_topk_workspace_bytes")
+            workspace = torch.empty(max(1, n.value), dtype=torch.uint8, device=self.device)
+        s = stream or torch.cuda.current_stream(self.device)
+        _check(lib().ckl_topk_cache(self._h, _ptr(H), _ptr(W), T, chunk, _ptr(idx), _ptr(logit),
+                                    _ptr(workspace), workspace.numel(),
+                                    ctypes.c_void_p(s.cuda_stream), int(sync)), "ckl_topk_cache")
+        return idx, logit
 
     def fwd_bwd_from_host(self, H_host, idx_host, logit_host, mask_host, staging, W, chunk,
                           out, workspace, stream=None) -> float:

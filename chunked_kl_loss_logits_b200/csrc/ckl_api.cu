@@ -48,11 +48,12 @@ struct ProfRec {
 
 enum KernelId {
   KID_MASK = 0, KID_GATHER, KID_LSE, KID_COMBINE, KID_GRAD, KID_SCALE, KID_FIXUP, KID_DH,
-  KID_DH_REDUCE, KID_DW, KID_LOSS, KID_COUNT
+  KID_DH_REDUCE, KID_DW, KID_LOSS, KID_TKMAX, KID_TKTHRESH, KID_TKEMIT, KID_TKSELECT, KID_COUNT
 };
 const char* kKernelNames[KID_COUNT] = {"mask_count", "teacher_topk", "lse_gemm", "lse_combine",
                                        "grad_gemm", "scale_e", "topk_fixup", "dh_gemm",
-                                       "dh_reduce", "dw_gemm", "loss_finalize"};
+                                       "dh_reduce", "dw_gemm", "loss_finalize", "cache_max_gemm",
+                                       "cache_threshold", "cache_emit_gemm", "cache_select"};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -366,9 +367,33 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
   return CKL_OK;
 }
 
+// Workspace of the teacher top-K cache builder for one chunk of Tc rows.
+struct TopkPlan {
+  int64_t Tc = 0;
+  int n_vt = 0;  // 256-wide vocabulary tiles
+  int cap = 0;   // candidates per row: at most K tiles can beat the threshold
+  size_t off_tbest = 0, off_theta = 0, off_cnt = 0, off_cand = 0, total = 0;
+};
+
+TopkPlan topk_plan(const ckl_ctx* h, int64_t T, int64_t chunk) {
+  TopkPlan p;
+  p.Tc = std::max<int64_t>(1, std::min(chunk, std::max<int64_t>(T, 1)));
+  p.n_vt = (int)((h->V + 255) / 256);
+  p.cap = (int)std::min<int64_t>(h->V, h->K * 256);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  p.off_tbest = take((size_t)p.n_vt * p.Tc * 8);
+  p.off_theta = take((size_t)p.Tc * 8);
+  p.off_cnt = take((size_t)p.Tc * 4);
+  p.off_cand = take((size_t)p.Tc * p.cap * 8);
+  p.total = o;
+  return p;
+}
+
 ckl_status fold_status(unsigned dev) {
   if (dev & ST_INDEX_RANGE) return CKL_ERR_INDEX_RANGE;
   if (dev & ST_TIMEOUT) return CKL_ERR_TIMEOUT;
+  if (dev & ST_INTERNAL) return CKL_ERR_INTERNAL;
   return CKL_OK;
 }
 
@@ -398,6 +423,7 @@ const char* ckl_status_str(ckl_status s) {
     case CKL_ERR_CUDA: return "CUDA runtime error";
     case CKL_ERR_TIMEOUT: return "device pipeline wait timed out";
     case CKL_ERR_ALIGNMENT: return "pointer misaligned";
+    case CKL_ERR_INTERNAL: return "internal consistency check failed";
   }
   return "unknown status";
 }
@@ -523,6 +549,77 @@ ckl_status ckl_sync_status(ckl_handle h, void* stream) {
 }
 
 int64_t ckl_launch_count(ckl_handle h) { return h ? h->launches : -1; }
+
+ckl_status ckl_topk_workspace_bytes(ckl_handle h, int64_t T, int64_t chunk, size_t* bytes) {
+  if (!h || !bytes || T < 0 || chunk < 1) return CKL_ERR_INVALID_ARG;
+  *bytes = topk_plan(h, T, chunk).total;
+  return CKL_OK;
+}
+
+ckl_status ckl_topk_cache(ckl_handle h, const void* H, const void* W, int64_t T, int64_t chunk,
+                          int32_t* topk_idx, float* topk_logit, void* workspace,
+                          size_t workspace_bytes, void* stream, int wait) {
+  if (!h || !W || T < 0 || chunk < 1 || chunk > h->max_chunk || chunk > INT32_MAX)
+    return CKL_ERR_INVALID_ARG;
+  if (T > 0 && (!H || !topk_idx || !topk_logit)) return CKL_ERR_INVALID_ARG;
+  if (h->dtype != CKL_BF16 || h->K > h->V) return CKL_ERR_UNSUPPORTED;
+  if (!aligned(W, 16) || (H && !aligned(H, 16)) || (topk_idx && !aligned(topk_idx, 4)) ||
+      (topk_logit && !aligned(topk_logit, 4)))
+    return CKL_ERR_ALIGNMENT;
+  const TopkPlan P = topk_plan(h, T, chunk);
+  if (T > 0 && (!workspace || !aligned(workspace, 256) || workspace_bytes < P.total))
+    return CKL_ERR_WORKSPACE;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return CKL_ERR_CUDA;
+  cudaGetLastError();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int V = (int)h->V, d = (int)h->d, K = (int)h->K;
+  unsigned char* base = static_cast<unsigned char*>(workspace);
+  float2* tbest = reinterpret_cast<float2*>(base + P.off_tbest);
+  float2* theta = reinterpret_cast<float2*>(base + P.off_theta);
+  int* cnt = reinterpret_cast<int*>(base + P.off_cnt);
+  float2* cand = reinterpret_cast<float2*>(base + P.off_cand);
+  Launcher L{h, s};
+  cudaError_t err = cudaSuccess;
+  auto chk = [&](cudaError_t e) { if (e != cudaSuccess && err == cudaSuccess) err = e; };
+  for (int64_t t0 = 0; t0 < T && err == cudaSuccess; t0 += chunk) {
+    const int Tc = (int)std::min<int64_t>(chunk, T - t0);
+    const double zflops = 2.0 * Tc * (double)V * d;
+    const unsigned char* Hc = static_cast<const unsigned char*>(H) + (size_t)t0 * d * 2;
+    TcMaps m;
+    if (!make_map(h, &m.a, Hc, d, Tc, (uint64_t)d * 2, 64, 128) ||
+        !make_map(h, &m.b, W, d, V, (uint64_t)d * 2, 64, 128))
+      return CKL_ERR_CUDA;
+    m.c = m.a;
+    chk(cudaMemsetAsync(cnt, 0, (size_t)Tc * 4, s));
+    chk(L(KID_TKMAX, zflops, 0, [&] {
+      TcLaunch p{};
+      p.kind = TcKind::TKMAX; p.M = Tc; p.N = V; p.n_kb = (d + 63) / 64; p.n_split = 1; p.V = V;
+      p.part = tbest; p.part_ld = Tc; p.status = h->d_status; p.num_sms = h->num_sms;
+      launch_tc(m, p, s);
+    }));
+    chk(L(KID_TKTHRESH, 0, (double)P.n_vt * Tc * 8, [&] {
+      launch_topk_threshold(tbest, P.n_vt, Tc, K, theta, s);
+    }));
+    chk(L(KID_TKEMIT, zflops, 0, [&] {
+      TcLaunch p{};
+      p.kind = TcKind::TKEMIT; p.M = Tc; p.N = V; p.n_kb = (d + 63) / 64; p.n_split = 1; p.V = V;
+      p.theta = theta; p.cand = cand; p.cand_cnt = cnt; p.cand_cap = P.cap;
+      p.status = h->d_status; p.num_sms = h->num_sms;
+      launch_tc(m, p, s);
+    }));
+    chk(L(KID_TKSELECT, 0, (double)Tc * K * 8, [&] {
+      launch_topk_select(cand, cnt, P.cap, Tc, K, topk_idx + t0 * K, topk_logit + t0 * K,
+                         h->d_status, s);
+    }));
+  }
+  if (err != cudaSuccess) {
+    std::fprintf(stderr, "ckl: CUDA error: %s\n", cudaGetErrorString(err));
+    return CKL_ERR_CUDA;
+  }
+  if (!wait) return CKL_OK;
+  return sync_and_read(h, s, nullptr, nullptr);
+}
 
 ckl_status ckl_set_recompute(ckl_handle h, int recompute) {
   if (!h) return CKL_ERR_INVALID_ARG;

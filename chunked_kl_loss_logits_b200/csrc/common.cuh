@@ -13,7 +13,7 @@
 namespace ckl {
 
 // Device status bits (folded into ckl_status by the host).
-enum : unsigned { ST_INDEX_RANGE = 1u, ST_TIMEOUT = 2u };
+enum : unsigned { ST_INDEX_RANGE = 1u, ST_TIMEOUT = 2u, ST_INTERNAL = 4u };
 
 // A wait gives up after this many SM cycles (about two seconds at 1.9 GHz); every
 // pipeline step of a correct run completes within microseconds.

@@ -380,6 +380,144 @@ __global__ void dh_reduce_bf16_kernel(const float* __restrict__ dHp, int n_split
   *reinterpret_cast<uint4*>(dH + e8) = o;
 }
 
+// ------------------------------------------------------------ teacher top-K cache
+// Candidates are ordered by (logit descending, id ascending), encoded in one
+// 64-bit key: the float's order-preserving bits above the complemented id.
+__device__ __forceinline__ unsigned long long topk_key(float v, int id) {
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)id);
+}
+__device__ __forceinline__ float topk_key_value(unsigned long long k) {
+  const uint32_t u = (uint32_t)(k >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+__device__ __forceinline__ int topk_key_id(unsigned long long k) {
+  return (int)(0xFFFFFFFFu - (uint32_t)k);
+}
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+constexpr int kThreshWarps = 8;
+constexpr int kThreshRegKeys = 32;  // keys per lane kept in registers (n_vt <= 1024)
+
+// Warp per row: the K-th best of the row's n_vt tile bests, by binary search on
+// the key bits (the largest key x with at least K keys >= x). Every one of the
+// row's K best logits is at least as good as it, and only the K tiles whose best
+// beats it can hold such logits, so at most K * 256 candidates follow.
+__global__ void __launch_bounds__(kThreshWarps * 32) topk_threshold_kernel(
+    const float2* __restrict__ tbest, int n_vt, int rows, int K, float2* __restrict__ theta) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kThreshWarps + warp;
+  if (i >= rows) return;
+  if (n_vt <= K) {  // every tile may hold top-K entries: take everything
+    if (lane == 0) theta[i] = make_float2(-INFINITY, __int_as_float(INT_MAX));
+    return;
+  }
+  const bool in_regs = n_vt <= 32 * kThreshRegKeys;
+  unsigned long long keys[kThreshRegKeys];
+#pragma unroll
+  for (int r = 0; r < kThreshRegKeys; ++r) {
+    const int j = r * 32 + lane;
+    keys[r] = 0;
+    if (in_regs && j < n_vt) {
+      const float2 b = tbest[(int64_t)j * rows + i];
+      keys[r] = topk_key(b.x, __float_as_int(b.y));
+    }
+  }
+  unsigned long long prefix = 0;
+  for (int bit = 63; bit >= 0; --bit) {
+    const unsigned long long cand = prefix | (1ull << bit);
+    int c = 0;
+    if (in_regs) {
+#pragma unroll
+      for (int r = 0; r < kThreshRegKeys; ++r) c += keys[r] >= cand;
+    } else {
+      for (int j = lane; j < n_vt; j += 32) {
+        const float2 b = tbest[(int64_t)j * rows + i];
+        c += topk_key(b.x, __float_as_int(b.y)) >= cand;
+      }
+    }
+    if (warp_sum_int(c) >= K) prefix = cand;
+  }
+  if (lane == 0) theta[i] = make_float2(topk_key_value(prefix), __int_as_float(topk_key_id(prefix)));
+}
+
+constexpr int kSelectThreads = 256;
+
+// Block per row: the K best of the row's candidates (by the same bit search over
+// the count of keys at least as good), then a bitonic sort into descending order.
+__global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(
+    const float2* __restrict__ cand, const int* __restrict__ cnt, int cap, int rows, int K,
+    int32_t* __restrict__ idx_out, float* __restrict__ logit_out, unsigned* status) {
+  __shared__ unsigned long long sel[1024];
+  __shared__ int wsum[kSelectThreads / 32];
+  __shared__ int nsel;
+  const int i = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int c = cnt[i];
+  if (c > cap) {  // cannot happen (at most K * 256 candidates); keep the first cap
+    if (tid == 0) atomicOr(status, (unsigned)ST_INTERNAL);
+    c = cap;
+  }
+  const float2* crow = cand + (int64_t)i * cap;
+  unsigned long long prefix = 0;
+  for (int bit = 63; bit >= 0; --bit) {
+    const unsigned long long want = prefix | (1ull << bit);
+    int n = 0;
+    for (int j = tid; j < c; j += kSelectThreads) {
+      const float2 e = crow[j];
+      n += topk_key(e.x, __float_as_int(e.y)) >= want;
+    }
+    n = warp_sum_int(n);
+    if (lane == 0) wsum[warp] = n;
+    __syncthreads();
+    int total = 0;
+#pragma unroll
+    for (int w = 0; w < kSelectThreads / 32; ++w) total += wsum[w];
+    __syncthreads();
+    if (total >= K) prefix = want;
+  }
+  int P = 1;
+  while (P < K) P <<= 1;
+  if (tid == 0) nsel = 0;
+  for (int j = tid; j < P; j += kSelectThreads) sel[j] = 0;  // padding sorts last
+  __syncthreads();
+  for (int j = tid; j < c; j += kSelectThreads) {
+    const float2 e = crow[j];
+    const unsigned long long k = topk_key(e.x, __float_as_int(e.y));
+    if (k >= prefix) {
+      const int slot = atomicAdd(&nsel, 1);
+      if (slot < K) sel[slot] = k;
+    }
+  }
+  __syncthreads();
+  // bitonic sort of sel[0, P) into descending key order
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int j = tid; j < P; j += kSelectThreads) {
+        const int partner = j ^ stride;
+        if (partner > j) {
+          const bool desc = (j & size) == 0;
+          const unsigned long long a = sel[j], b = sel[partner];
+          if (desc ? (a < b) : (a > b)) {
+            sel[j] = b;
+            sel[partner] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int k = tid; k < K; k += kSelectThreads) {
+    idx_out[(int64_t)i * K + k] = topk_key_id(sel[k]);
+    logit_out[(int64_t)i * K + k] = topk_key_value(sel[k]);
+  }
+}
+
 constexpr int kReduceThreads = 1024;
 
 __device__ double block_sum_d(double v, double* sh) {
@@ -491,6 +629,18 @@ template void launch_fixup<uint16_t>(const int32_t*, int64_t, int, int, int, int
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
                            cudaStream_t s) {
   dh_reduce_bf16_kernel<<<blocks_for(n_elem / 8, 256), 256, 0, s>>>(dHp, n_split, n_elem, dH);
+}
+
+void launch_topk_threshold(const float2* tbest, int n_vt, int rows, int K, float2* theta,
+                           cudaStream_t s) {
+  topk_threshold_kernel<<<blocks_for(rows, kThreshWarps), kThreshWarps * 32, 0, s>>>(
+      tbest, n_vt, rows, K, theta);
+}
+
+void launch_topk_select(const float2* cand, const int* cnt, int cap, int rows, int K,
+                        int32_t* idx_out, float* logit_out, unsigned* status, cudaStream_t s) {
+  topk_select_kernel<<<rows, kSelectThreads, 0, s>>>(cand, cnt, cap, rows, K, idx_out, logit_out,
+                                                     status);
 }
 
 void launch_loss_finalize(const float* ell_all, const uint8_t* mask, int64_t T, Misc* misc,

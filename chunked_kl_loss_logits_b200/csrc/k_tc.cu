@@ -15,6 +15,9 @@
 //         reduced in a fixed order afterwards).
 //   DW  : dW (+)= G^T H_c, contraction over the chunk's tokens; the epilogue adds
 //         its fp32 tile into dW with a TMA reduce-add (the add happens in L2).
+//   TKMAX, TKEMIT: the teacher top-K cache builder's two passes over the
+//         teacher's logits (best logit per row and tile; candidates at least as
+//         good as the row's threshold), same mainloop as LSE.
 //
 // Work unit: a 256 x BN output tile computed by a CTA pair (a cluster of two
 // CTAs on neighbouring SMs) with tcgen05.mma.cta_group::2: each CTA stages its
@@ -63,6 +66,8 @@ template <> struct Cfg<TcKind::LSE>  { static constexpr int BN = 256; static con
 template <> struct Cfg<TcKind::GRAD> { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
 template <> struct Cfg<TcKind::DH>   { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = true;  static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
 template <> struct Cfg<TcKind::DW>   { static constexpr int BN = 256; static constexpr bool A_MN = true,  B_MN = true;  static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::TKMAX>  { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
+template <> struct Cfg<TcKind::TKEMIT> { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
 
 template <TcKind KIND>
 struct Layout {
@@ -414,6 +419,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             stage_and_issue(ch, cb, row0, false);
           }
         }
+      } else if constexpr (KIND == TcKind::TKMAX) {
+        // the row's best logit in this vocabulary tile and its smallest id
+        float best = -INFINITY;
+        int bid = INT_MAX;
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          float v[32];
+          tmem_ld32(taddr + cc * 32, v);
+          const int cb = col0 + cc * 32;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (cb + j < p.V && v[j] > best) { best = v[j]; bid = cb + j; }
+        }
+        if (row_ok) p.part[(int64_t)c.nt * p.part_ld + grow] = make_float2(best, __int_as_float(bid));
+      } else if constexpr (KIND == TcKind::TKEMIT) {
+        // every (logit, id) at least as good as the row's threshold joins its candidates
+        float tv = INFINITY;
+        int tid = -1;
+        if (row_ok) {
+          const float2 th = p.theta[grow];
+          tv = th.x;
+          tid = __float_as_int(th.y);
+        }
+        int* cnt = p.cand_cnt + grow;
+        float2* crow = p.cand + (int64_t)grow * p.cand_cap;
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          float v[32];
+          tmem_ld32(taddr + cc * 32, v);
+          const int cb = col0 + cc * 32;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int col = cb + j;
+            if (col < p.V && (v[j] > tv || (v[j] == tv && col <= tid))) {
+              const int slot = atomicAdd(cnt, 1);
+              if (slot < p.cand_cap) crow[slot] = make_float2(v[j], __int_as_float(col));
+            }
+          }
+        }
       } else if constexpr (KIND == TcKind::DH) {
         // fp32 partial of split c.split, plain vector stores
         float* out = p.dHp + (int64_t)c.split * p.M * p.N + (int64_t)grow * p.N;
@@ -510,6 +554,8 @@ int tc_bn(TcKind k) {
     case TcKind::LSE: return Cfg<TcKind::LSE>::BN;
     case TcKind::GRAD: return Cfg<TcKind::GRAD>::BN;
     case TcKind::DH: return Cfg<TcKind::DH>::BN;
+    case TcKind::TKMAX: return Cfg<TcKind::TKMAX>::BN;
+    case TcKind::TKEMIT: return Cfg<TcKind::TKEMIT>::BN;
     default: return Cfg<TcKind::DW>::BN;
   }
 }
@@ -519,6 +565,8 @@ cudaError_t launch_tc(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
     case TcKind::LSE: return launch_kind<TcKind::LSE>(maps, p, s);
     case TcKind::GRAD: return launch_kind<TcKind::GRAD>(maps, p, s);
     case TcKind::DH: return launch_kind<TcKind::DH>(maps, p, s);
+    case TcKind::TKMAX: return launch_kind<TcKind::TKMAX>(maps, p, s);
+    case TcKind::TKEMIT: return launch_kind<TcKind::TKEMIT>(maps, p, s);
     default: return launch_kind<TcKind::DW>(maps, p, s);
   }
 }

@@ -56,6 +56,13 @@ void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int64_t 
 void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s);
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
                            cudaStream_t s);
+// Teacher top-K cache: per row, the threshold = the K-th best of the n_vt tile
+// bests (logit descending, id ascending), or "take everything" when n_vt <= K.
+void launch_topk_threshold(const float2* tbest, int n_vt, int rows, int K, float2* theta,
+                           cudaStream_t s);
+// Per row, the K best candidates in descending order -> idx, logit (row stride K).
+void launch_topk_select(const float2* cand, const int* cnt, int cap, int rows, int K,
+                        int32_t* idx_out, float* logit_out, unsigned* status, cudaStream_t s);
 void launch_loss_finalize(const float* ell_all, const uint8_t* mask, int64_t T, Misc* misc,
                           float* loss, cudaStream_t s);
 
@@ -74,7 +81,7 @@ constexpr int kSimtTile = 64;
 struct TcMaps {
   CUtensorMap a, b, c;  // operands A and B; c = epilogue store target (G or dW)
 };
-enum class TcKind : int { LSE = 0, GRAD = 1, DH = 2, DW = 3 };
+enum class TcKind : int { LSE = 0, GRAD = 1, DH = 2, DW = 3, TKMAX = 4, TKEMIT = 5 };
 struct TcLaunch {
   TcKind kind;
   int M, N, n_kb;  // output rows, output cols, 64-wide blocks along the contraction
@@ -93,6 +100,13 @@ struct TcLaunch {
   float* dHp;         // DH
   float* dW;          // DW
   int first;          // DW: overwrite instead of accumulate
+  // teacher top-K cache: TKMAX writes each row's best (logit, id) per vocabulary
+  // tile into `part` (id stored as float bits); TKEMIT appends every (logit, id)
+  // at least as good as the row's threshold `theta` to the row's candidate list.
+  const float2* theta;
+  float2* cand;
+  int* cand_cnt;
+  int cand_cap;
   unsigned* status;
   int num_sms;
 };

@@ -61,7 +61,8 @@ typedef enum {
   CKL_ERR_INDEX_RANGE = 4,  /* device: a topk_idx entry outside [0, V) */
   CKL_ERR_CUDA = 5,         /* a CUDA runtime call failed (no device, launch failure, ...) */
   CKL_ERR_TIMEOUT = 6,      /* device: a pipeline wait exceeded its bound; the kernel gave up */
-  CKL_ERR_ALIGNMENT = 7     /* a pointer is not aligned as stated above */
+  CKL_ERR_ALIGNMENT = 7,    /* a pointer is not aligned as stated above */
+  CKL_ERR_INTERNAL = 8      /* device: an internal consistency check failed */
 } ckl_status;
 
 typedef enum { CKL_F32 = 0, CKL_BF16 = 1 } ckl_dtype;
@@ -146,6 +147,27 @@ ckl_status ckl_forward_static(int device, ckl_dtype dtype, int64_t V, int64_t d,
                               const float* topk_logit, const uint8_t* mask, int64_t T,
                               int64_t chunk, float* loss, float* token_lse, float* token_loss,
                               void* stream, float* loss_host);
+
+/* Teacher top-K cache builder: the offline half of the method ("Efficient
+ * Knowledge Distillation for LLMs: Offline Top-K Logits and a Fused Chunked KL
+ * Loss", abstract; the author's forum post: the teacher runs once and each
+ * position keeps its 100 largest logits). For a handle made with the TEACHER's
+ * shape (V, d = teacher hidden size, K = cache width; bf16 only, K <= V):
+ * H (T x d, device) holds the teacher's last hidden states and W (V x d,
+ * device) its LM head. Writes, per token, the K largest logits of H_t W^T
+ * (fp32, from a bf16 x bf16 -> fp32 contraction) to topk_logit (T x K) and their
+ * ids to topk_idx (T x K), in descending order of logit; equal logits in
+ * ascending id order. These are exactly the topk_idx / topk_logit inputs of
+ * ckl_fwd_bwd. Processed `chunk` tokens at a time (1 <= chunk <= max_chunk) with
+ * two tensor-core passes over the logits (best per 256-column tile, then the
+ * candidates at least as good as the K-th best tile best) and a per-token
+ * selection; the workspace is ckl_topk_workspace_bytes bytes (about
+ * chunk * min(V, 256 K) * 8 bytes). wait != 0: wait for the stream and return
+ * the device-detected status. */
+ckl_status ckl_topk_workspace_bytes(ckl_handle h, int64_t T, int64_t chunk, size_t* bytes);
+ckl_status ckl_topk_cache(ckl_handle h, const void* H, const void* W, int64_t T, int64_t chunk,
+                          int32_t* topk_idx, float* topk_logit, void* workspace,
+                          size_t workspace_bytes, void* stream, int wait);
 
 /* Wait for `stream` and return the device-detected status of the calls enqueued
  * on it since the last synchronising call (clears it). */

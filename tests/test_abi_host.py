@@ -26,7 +26,7 @@ def test_exports_every_declared_function(L):
 
 
 def test_status_strings(L):
-    for code in range(8):
+    for code in range(9):
         s = L.ckl_status_str(code)
         assert s and s != b"unknown status"
     assert L.ckl_status_str(99) == b"unknown status"
