@@ -427,6 +427,113 @@ def run_sweep(args, w):
         h.close()
 
 
+def _dense_kl(H, W, idx, logit):
+    """Full Dense KL in plain PyTorch: the cached top-K probabilities scattered into
+    a T x V teacher, compared with the student's dense log-softmax (autograd)."""
+    import torch
+    z = H @ W.t()
+    logq = torch.log_softmax(z.float(), dim=-1)
+    P = torch.zeros_like(logq).scatter_add_(1, idx.long(), torch.softmax(logit.float(), dim=-1))
+    return torch.nn.functional.kl_div(logq, P, reduction="sum") / H.shape[0]
+
+
+def _forward_chunked_kl(H, W, idx, logit, chunk):
+    """Forward-Chunked Loss in plain PyTorch: sparse teacher, the loss evaluated in
+    sequence chunks, but the full student logits come from one projection and
+    autograd keeps them for the backward."""
+    import torch
+    z = H @ W.t()
+    total = z.new_zeros((), dtype=torch.float32)
+    for t0 in range(0, H.shape[0], chunk):
+        zc = z[t0:t0 + chunk].float()
+        lp = torch.log_softmax(logit[t0:t0 + chunk], dim=-1)
+        p = lp.exp()
+        lse = torch.logsumexp(zc, dim=-1)
+        zk = zc.gather(1, idx[t0:t0 + chunk].long())
+        total = total + (p * lp).sum() - (p * zk).sum() + lse.sum()
+    return total / H.shape[0]
+
+
+def run_compare(args, w):
+    """The pages' two other loss forms, in plain PyTorch on this GPU, beside this library.
+
+    For T in a range of sequence lengths on the workload's (V, d, K): peak device
+    memory above the inputs and mean forward + backward time of each form, one JSON
+    line per (method, T). A form whose estimated footprint exceeds the memory
+    budget is not run (reported as skipped); an out-of-memory exception is
+    reported, not raised. Inputs are the workload's own (distinct teacher ids, so
+    the dense scatter and the sparse forms agree).
+    """
+    import torch
+
+    from chunked_kl_loss_logits_b200 import ckl
+    from chunked_kl_loss_logits_b200.workloads import make_inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    chunk = args.chunk or w.chunk
+    free, total = torch.cuda.mem_get_info(dev)
+    budget = 0.8 * free
+    for T in args.compare_tokens:
+        x = make_inputs(w, T=T)
+        H0 = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
+        W0 = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+        idx = torch.from_numpy(x["idx"]).to(dev)
+        lg = torch.from_numpy(x["logit"]).to(dev)
+        del x
+        # bytes held at the peak: bf16 z and its grad, several fp32 T x V tensors
+        est = {"dense_kl": T * w.V * (2 * 2 + 4 * 4), "forward_chunked": T * w.V * (2 * 2 + 4 * 2),
+               "ckl": 0}
+        for method in ("dense_kl", "forward_chunked", "ckl"):
+            rec = {"kind": "compare", "method": method, "workload": w.name, "T": T, "V": w.V,
+                   "d": w.d, "K": w.K, "chunk": chunk if method != "dense_kl" else None}
+            if est[method] > budget:
+                rec["status"] = "skipped: estimated %.0f GiB above the %.0f GiB budget" % (
+                    est[method] / 2**30, budget / 2**30)
+                print(json.dumps(rec), flush=True)
+                continue
+            H = H0.clone().requires_grad_(method != "ckl")
+            W = W0.clone().requires_grad_(method != "ckl")
+            h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=chunk, device=dev) if method == "ckl" else None
+
+            def step():
+                if method == "ckl":
+                    return h.fwd_bwd(H, W, idx, lg, None, chunk=chunk, sync=False)[0]
+                H.grad = W.grad = None
+                loss = _dense_kl(H, W, idx, lg) if method == "dense_kl" else \
+                    _forward_chunked_kl(H, W, idx, lg, chunk)
+                loss.backward()
+                return loss.detach()
+
+            try:
+                torch.cuda.synchronize(dev)
+                torch.cuda.empty_cache()
+                base = torch.cuda.memory_allocated(dev)
+                torch.cuda.reset_peak_memory_stats(dev)
+                loss = step()
+                torch.cuda.synchronize(dev)
+                peak = torch.cuda.max_memory_allocated(dev) - base
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                n = args.compare_steps
+                e0.record()
+                for _ in range(n):
+                    loss = step()
+                e1.record()
+                torch.cuda.synchronize(dev)
+                ms = e0.elapsed_time(e1) / n
+                rec.update(status="ok", loss=float(loss), peak_gib_above_inputs=peak / 2**30,
+                           ms_per_step=ms, tokens_per_s=T / (ms / 1e3),
+                           tflops_useful=6.0 * T * w.V * w.d / (ms / 1e3) / 1e12)
+            except torch.cuda.OutOfMemoryError as e:
+                rec["status"] = "out of memory: " + str(e).splitlines()[0][:120]
+            print(json.dumps(rec), flush=True)
+            del H, W
+            if h is not None:
+                h.close()
+            torch.cuda.synchronize(dev)
+            torch.cuda.empty_cache()
+        del H0, W0, idx, lg
+
+
 def run_topk_cache(args, w):
     """Teacher top-K cache builder on one workload's shape: tokens/s of one cache pass.
 
@@ -488,6 +595,12 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="256K workload: throughput vs chunk and peak memory vs T (extra JSON lines)")
     ap.add_argument("--sweep-steps", type=int, default=3)
+    ap.add_argument("--compare", action="store_true",
+                    help="the pages' Full Dense KL and Forward-Chunked Loss in plain PyTorch beside "
+                         "this library: peak memory and step time vs T (extra JSON lines)")
+    ap.add_argument("--compare-tokens", type=lambda v: [int(t) for t in v.split(",")],
+                    default=[4096, 8192, 16384, 32768])
+    ap.add_argument("--compare-steps", type=int, default=3)
     ap.add_argument("--topk-cache", action="store_true",
                     help="time the teacher top-K cache builder on the workload's shape instead")
     ap.add_argument("--recompute", action="store_true",
@@ -512,6 +625,9 @@ def main():
         return
     if args.topk_cache:
         run_topk_cache(args, w)
+        return
+    if args.compare:
+        run_compare(args, w)
         return
     if world > 1:
         import datetime

@@ -14,19 +14,34 @@ import re
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "lib", "libckl.so")
+# The in-tree build; CKL_LIBRARY names another build of the same library.
+LIB_PATH = os.environ.get("CKL_LIBRARY") or os.path.join(_PKG, "lib", "libckl.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "ckl.h")
 
 F32, BF16 = 0, 1
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported size", 3: "workspace",
            4: "top-K index out of range", 5: "CUDA error", 6: "device wait timed out",
-           7: "pointer misaligned", 8: "internal consistency check failed"}
+           7: "pointer misaligned", 8: "internal consistency check failed",
+           9: "a caller-supplied collective failed"}
 
 
 class CKLError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: {_STATUS.get(code, code)} (status {code})")
         self.code = code
+
+
+_GatherFn = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                             ctypes.c_int64, ctypes.c_void_p)
+_ReduceFn = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                             ctypes.c_void_p)
+
+
+class _VocabGroupC(ctypes.Structure):
+    """Mirror of ckl_vocab_group."""
+    _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("V_total", ctypes.c_int64),
+                ("v0", ctypes.c_int64), ("all_gather", _GatherFn), ("all_reduce_sum", _ReduceFn),
+                ("user", ctypes.c_void_p)]
 
 
 class KernelStat(ctypes.Structure):
@@ -65,6 +80,10 @@ def lib() -> ctypes.CDLL:
         "ckl_set_recompute": ([_P, ctypes.c_int], ctypes.c_int),
         "ckl_topk_workspace_bytes": ([_P, _I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
         "ckl_topk_cache": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _SZ, _P, ctypes.c_int], ctypes.c_int),
+        "ckl_vp_workspace_bytes": ([_P, ctypes.c_int32, _I64, _I64, ctypes.POINTER(_SZ)],
+                                   ctypes.c_int),
+        "ckl_fwd_bwd_vocab_parallel": ([_P, ctypes.POINTER(_VocabGroupC), _P, _P, _P, _P, _P, _I64,
+                                        _I64, _P, _P, _P, _P, _P, _P, _SZ, _P, _P], ctypes.c_int),
         "ckl_profile_enable": ([_P, ctypes.c_int, ctypes.c_int], ctypes.c_int),
         "ckl_profile_collect": ([_P, ctypes.POINTER(KernelStat), ctypes.c_int,
                                  ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -91,6 +110,85 @@ def _ptr(t):
 def _check(code: int, what: str):
     if code != 0:
         raise CKLError(code, what)
+
+
+class _DevArray:
+    """A raw device pointer seen as a float32 vector (CUDA array interface, no copy)."""
+
+    def __init__(self, ptr: int, count: int):
+        self.__cuda_array_interface__ = {"shape": (count,), "typestr": "<f4",
+                                         "data": (ptr, False), "version": 3, "stream": None}
+
+
+def vocab_shards(V_total: int, world: int, align: int = 256) -> list:
+    """(v0, V_r) of each rank: contiguous row ranges of the LM head, as equal as
+    possible in whole `align`-row blocks (the last rank takes the remainder)."""
+    if world < 1 or V_total < world:
+        raise ValueError("need 1 <= world <= V_total")
+    blocks = (V_total + align - 1) // align
+    out, v0 = [], 0
+    for r in range(world):
+        nb = blocks // world + (1 if r < blocks % world else 0)
+        v1 = min(V_total, v0 + nb * align) if r < world - 1 else V_total
+        out.append((v0, v1 - v0))
+        v0 = v1
+    if any(n <= 0 for _, n in out):
+        raise ValueError("a rank would hold no rows")
+    return out
+
+
+class VocabGroup:
+    """This rank's place in a vocabulary-parallel group and the group's two collectives.
+
+    all_gather(send, recv): send is a float32 vector of n entries, recv one of
+    world * n entries to fill rank-major; all_reduce_sum(buf): in place. Both
+    get device tensors and must be ordered on the current CUDA stream (the
+    library's stream is made current around each call) and return None.
+    """
+
+    def __init__(self, world: int, rank: int, V_total: int, v0: int, all_gather, all_reduce_sum):
+        self.world, self.rank, self.V_total, self.v0 = world, rank, V_total, v0
+        self.all_gather, self.all_reduce_sum = all_gather, all_reduce_sum
+        self.error = None
+
+    def _c(self, device):
+        def as_stream(ptr):
+            return torch.cuda.ExternalStream(ptr, device=device) if ptr else \
+                torch.cuda.default_stream(device)
+
+        def gather(_user, send, recv, count, stream):
+            try:
+                with torch.cuda.stream(as_stream(stream)):
+                    a = torch.as_tensor(_DevArray(send, count), device=device)
+                    b = torch.as_tensor(_DevArray(recv, count * self.world), device=device)
+                    self.all_gather(a, b)
+                return 0
+            except Exception as e:  # reported as CKL_ERR_COLLECTIVE; kept for the caller
+                self.error = e
+                return 1
+
+        def reduce(_user, buf, count, stream):
+            try:
+                with torch.cuda.stream(as_stream(stream)):
+                    self.all_reduce_sum(torch.as_tensor(_DevArray(buf, count), device=device))
+                return 0
+            except Exception as e:
+                self.error = e
+                return 1
+
+        fns = (_GatherFn(gather), _ReduceFn(reduce))  # kept alive by the caller for the call
+        return _VocabGroupC(self.world, self.rank, self.V_total, self.v0, fns[0], fns[1], None), fns
+
+
+def torch_vocab_group(V_total: int, group=None) -> VocabGroup:
+    """A VocabGroup over a torch.distributed process group (NCCL on GPUs): this
+    rank's rows come from vocab_shards(V_total, world)."""
+    import torch.distributed as dist
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    v0, _ = vocab_shards(V_total, world)[rank]
+    return VocabGroup(world, rank, V_total, v0,
+                      lambda send, recv: dist.all_gather_into_tensor(recv, send, group=group),
+                      lambda buf: dist.all_reduce(buf, group=group))
 
 
 class ChunkedKL:
@@ -217,6 +315,40 @@ class ChunkedKL:
                                  ctypes.c_void_p(s.cuda_stream),
                                  ctypes.byref(host) if sync else None), "ckl_forward")
         return (loss, lse, ell) if token_stats else loss
+
+    def fwd_bwd_vocab_parallel(self, group: VocabGroup, H, W_shard, idx, logit, mask=None,
+                               chunk: int | None = None, token_stats: bool = False,
+                               sync: bool = True, stream=None):
+        """Loss, dH (full, identical on every rank) and dW_shard (this rank's V x d rows).
+
+        The handle's V is this rank's row count; ids are global in [0, group.V_total).
+        """
+        T = self._inputs(H, W_shard, idx, logit, mask)
+        chunk = min(chunk or self.max_chunk, self.max_chunk)
+        n = _SZ()
+        _check(lib().ckl_vp_workspace_bytes(self._h, group.world, T, chunk, ctypes.byref(n)),
+               "ckl_vp_workspace_bytes")
+        ws = torch.empty(max(1, n.value), dtype=torch.uint8, device=self.device)
+        loss = torch.empty((), dtype=torch.float32, device=self.device)
+        dH = torch.empty_like(H)
+        dW = torch.empty((self.V, self.d), dtype=torch.float32, device=self.device)
+        lse = ell = None
+        if token_stats:
+            lse = torch.empty(T, dtype=torch.float32, device=self.device)
+            ell = torch.empty(T, dtype=torch.float32, device=self.device)
+        s = stream or torch.cuda.current_stream(self.device)
+        g, keep = group._c(self.device)
+        host = ctypes.c_float() if sync else None
+        group.error = None
+        code = lib().ckl_fwd_bwd_vocab_parallel(
+            self._h, ctypes.byref(g), _ptr(H), _ptr(W_shard), _ptr(idx), _ptr(logit), _ptr(mask),
+            T, chunk, _ptr(loss), _ptr(dH), _ptr(dW), _ptr(lse), _ptr(ell), _ptr(ws), ws.numel(),
+            ctypes.c_void_p(s.cuda_stream), ctypes.byref(host) if sync else None)
+        del keep
+        if code == 9 and group.error is not None:
+            raise CKLError(code, "ckl_fwd_bwd_vocab_parallel") from group.error
+        _check(code, "ckl_fwd_bwd_vocab_parallel")
+        return (loss, dH, dW, lse, ell) if token_stats else (loss, dH, dW)
 
     def topk_cache(self, H, W, chunk: int | None = None, workspace=None, sync: bool = True,
                    stream=None):

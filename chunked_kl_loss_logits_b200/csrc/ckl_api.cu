@@ -48,12 +48,15 @@ struct ProfRec {
 
 enum KernelId {
   KID_MASK = 0, KID_GATHER, KID_LSE, KID_COMBINE, KID_GRAD, KID_SCALE, KID_FIXUP, KID_DH,
-  KID_DH_REDUCE, KID_DW, KID_LOSS, KID_TKMAX, KID_TKTHRESH, KID_TKEMIT, KID_TKSELECT, KID_COUNT
+  KID_DH_REDUCE, KID_DW, KID_LOSS, KID_TKMAX, KID_TKTHRESH, KID_TKEMIT, KID_TKSELECT,
+  KID_VP_MERGE, KID_DH_F32, KID_TO_BF16, KID_VP_GATHER, KID_VP_REDUCE, KID_COUNT
 };
 const char* kKernelNames[KID_COUNT] = {"mask_count", "teacher_topk", "lse_gemm", "lse_combine",
                                        "grad_gemm", "scale_e", "topk_fixup", "dh_gemm",
                                        "dh_reduce", "dw_gemm", "loss_finalize", "cache_max_gemm",
-                                       "cache_threshold", "cache_emit_gemm", "cache_select"};
+                                       "cache_threshold", "cache_emit_gemm", "cache_select",
+                                       "vp_merge", "dh_reduce_f32", "dh_to_bf16",
+                                       "vp_all_gather", "vp_all_reduce"};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -100,6 +103,8 @@ struct WsPlan {
   size_t off_ell = 0, off_lse = 0, off_misc = 0, off_tok = 0, off_cst = 0, off_zk = 0,
          off_Pk = 0, off_part = 0, off_xpart = 0, off_sid = 0, off_sp = 0, off_G = 0, off_dHp = 0,
          total = 0;
+  // vocabulary split over ranks: this rank's stats, the gathered stats, dH_c in fp32
+  size_t off_stats = 0, off_stats_all = 0, off_dhf = 0;
 };
 
 // dH tiles are 256 x 256 outputs computed by CTA pairs; split the vocabulary
@@ -120,7 +125,7 @@ int pick_dh_split(int64_t Tc, int64_t d, int64_t V, int num_sms) {
   return (int)((n_kb + kps - 1) / kps);
 }
 
-WsPlan plan(const ckl_ctx* h, int64_t T, int64_t chunk, bool backward) {
+WsPlan plan(const ckl_ctx* h, int64_t T, int64_t chunk, bool backward, int world = 0) {
   WsPlan p;
   p.Tc = std::max<int64_t>(1, std::min(chunk, std::max<int64_t>(T, 1)));
   const bool bf16 = h->dtype == CKL_BF16;
@@ -146,6 +151,11 @@ WsPlan plan(const ckl_ctx* h, int64_t T, int64_t chunk, bool backward) {
   if (backward) {
     p.off_G = take((size_t)p.Tc * p.ldG * (bf16 ? 2 : 4));
     if (bf16) p.off_dHp = take((size_t)p.n_split * p.Tc * h->d * 4);
+  }
+  if (world > 0) {
+    p.off_stats = take((size_t)p.Tc * 16);
+    p.off_stats_all = take((size_t)world * p.Tc * 16);
+    p.off_dhf = take((size_t)p.Tc * h->d * 4);
   }
   p.total = o;
   return p;
@@ -189,6 +199,21 @@ struct Launcher {
     h->launches++;
     return e;
   }
+  // A caller-supplied collective: profiled under `kid`, not counted as a launch.
+  template <class F>
+  int collective(int kid, double bytes, F&& f) {
+    int slot = -1;
+    if (h->prof && h->ev_used * 2 + 1 < (int)h->ev.size()) {
+      slot = h->ev_used++;
+      cudaEventRecord(h->ev[2 * slot], s);
+    }
+    const int rc = f();
+    if (slot >= 0) {
+      cudaEventRecord(h->ev[2 * slot + 1], s);
+      h->recs.push_back(ProfRec{kid, slot, 0.0, bytes});
+    }
+    return rc;
+  }
 };
 
 ckl_status check_common(const ckl_ctx* h, const void* H, const void* W, const int32_t* idx,
@@ -203,10 +228,11 @@ ckl_status check_common(const ckl_ctx* h, const void* H, const void* W, const in
   return CKL_OK;
 }
 
+// `group` (vocabulary split over ranks, bf16 backward only) or nullptr.
 ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, const float* logit,
                const uint8_t* mask, int64_t T, int64_t chunk, float* loss, void* dH, float* dW,
                float* tok_lse, float* tok_loss, void* ws, size_t ws_bytes, cudaStream_t s,
-               bool backward) {
+               bool backward, const ckl_vocab_group* group = nullptr) {
   ckl_status st = check_common(h, H, W, idx, logit, T, chunk, loss);
   if (st != CKL_OK) return st;
   if (backward) {
@@ -215,7 +241,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
   }
   if ((tok_lse && !aligned(tok_lse, 4)) || (tok_loss && !aligned(tok_loss, 4)))
     return CKL_ERR_ALIGNMENT;
-  const WsPlan P = plan(h, T, chunk, backward);
+  const WsPlan P = plan(h, T, chunk, backward, group ? group->world : 0);
   if (!ws || !aligned(ws, 256) || ws_bytes < P.total) return CKL_ERR_WORKSPACE;
 
   DeviceGuard guard(h->device);
@@ -237,6 +263,12 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
   b.dHp = (backward && h->dtype == CKL_BF16) ? reinterpret_cast<float*>(base + P.off_dHp) : nullptr;
   float* ell_all = reinterpret_cast<float*>(base + P.off_ell);
   float* lse_all = reinterpret_cast<float*>(base + P.off_lse);
+  float4* stats = group ? reinterpret_cast<float4*>(base + P.off_stats) : nullptr;
+  float4* stats_all = group ? reinterpret_cast<float4*>(base + P.off_stats_all) : nullptr;
+  float* dhf = group ? reinterpret_cast<float*>(base + P.off_dhf) : nullptr;
+  const int V_all = group ? (int)group->V_total : (int)h->V;
+  const int v0 = group ? (int)group->v0 : 0;
+  int coll_rc = 0;  // first failing collective's return code
 
   const int V = (int)h->V, d = (int)h->d, K = (int)h->K;
   const bool bf16 = h->dtype == CKL_BF16;
@@ -248,14 +280,30 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
   chk(L(KID_MASK, 0, (double)T, [&] { launch_mask_count(mask, T, b.misc, s); }));
   if (backward && T == 0) chk(cudaMemsetAsync(dW, 0, (size_t)V * d * 4, s));
 
-  for (int64_t t0 = 0; t0 < T && err == cudaSuccess; t0 += chunk) {
+  // With a group every chunk makes its two collectives even after an error (the
+  // ranks' calls must stay matched); only the kernels are skipped.
+  for (int64_t t0 = 0; t0 < T && (err == cudaSuccess || group); t0 += chunk) {
     const int Tc = (int)std::min<int64_t>(chunk, T - t0);
     const double zflops = 2.0 * Tc * (double)V * d;
     const unsigned char* Hc = static_cast<const unsigned char*>(H) + (size_t)t0 * d * esz;
+    if (err != cudaSuccess || coll_rc != 0) {
+      if (!coll_rc) {
+        coll_rc = L.collective(KID_VP_GATHER, 0, [&] {
+          return group->all_gather(group->user, reinterpret_cast<const float*>(stats),
+                                   reinterpret_cast<float*>(stats_all), (int64_t)Tc * 4, s);
+        });
+      }
+      if (!coll_rc) {
+        coll_rc = L.collective(KID_VP_REDUCE, 0, [&] {
+          return group->all_reduce_sum(group->user, dhf, (int64_t)Tc * d, s);
+        });
+      }
+      continue;
+    }
 
     if (bf16) {
       chk(L(KID_GATHER, 0, (double)Tc * K * 16.0, [&] {
-        launch_teacher(idx, logit, t0, Tc, V, K, b, h->d_status, s);
+        launch_teacher(idx, logit, t0, Tc, V_all, v0, K, b, h->d_status, s);
       }));
     } else {
       chk(L(KID_GATHER, 2.0 * Tc * K * d, (double)Tc * (K * 8.0 + d * esz + K * d * esz), [&] {
@@ -290,8 +338,20 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
       }
     }));
     chk(L(KID_COMBINE, 0, (double)P.n_vt * Tc * 8, [&] {
-      launch_combine(t0, Tc, P.n_vt, mask, b, lse_all, ell_all, s);
+      launch_combine(t0, Tc, P.n_vt, mask, b, lse_all, ell_all, stats, s);
     }));
+    if (group) {
+      // this rank's (max, sum, cross) per token to every rank; merged in rank order
+      if (!coll_rc) {
+        coll_rc = L.collective(KID_VP_GATHER, (double)group->world * Tc * 16, [&] {
+          return group->all_gather(group->user, reinterpret_cast<const float*>(stats),
+                                   reinterpret_cast<float*>(stats_all), (int64_t)Tc * 4, s);
+        });
+      }
+      chk(L(KID_VP_MERGE, 0, (double)Tc * (group->world * 16.0 + 24.0), [&] {
+        launch_vp_merge(t0, Tc, group->world, stats_all, mask, b, lse_all, ell_all, s);
+      }));
+    }
     if (!backward) continue;
 
     if (store_e) {
@@ -313,8 +373,8 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
       }));
     }
     chk(L(KID_FIXUP, 0, (double)Tc * K * (12.0 + 2 * esz), [&] {
-      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, P.ldG, b, false, s);
-      else launch_fixup<float>(idx, t0, Tc, K, V, P.ldG, b, false, s);
+      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, v0, P.ldG, b, false, s);
+      else launch_fixup<float>(idx, t0, Tc, K, V, v0, P.ldG, b, false, s);
     }));
 
     unsigned char* dHc = static_cast<unsigned char*>(dH) + (size_t)t0 * d * esz;
@@ -333,10 +393,25 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
         p.dHp = b.dHp; p.status = h->d_status; p.num_sms = h->num_sms;
         launch_tc(mh, p, s);
       }));
-      chk(L(KID_DH_REDUCE, 0, (double)Tc * d * (4.0 * P.n_split + 2.0), [&] {
-        launch_dh_reduce_bf16(b.dHp, P.n_split, (int64_t)Tc * d, reinterpret_cast<uint16_t*>(dHc),
-                              s);
-      }));
+      if (!group) {
+        chk(L(KID_DH_REDUCE, 0, (double)Tc * d * (4.0 * P.n_split + 2.0), [&] {
+          launch_dh_reduce_bf16(b.dHp, P.n_split, (int64_t)Tc * d,
+                                reinterpret_cast<uint16_t*>(dHc), s);
+        }));
+      } else {
+        // this rank's share of dH_c in fp32, summed over ranks, then bf16
+        chk(L(KID_DH_F32, 0, (double)Tc * d * (4.0 * P.n_split + 4.0), [&] {
+          launch_dh_reduce_f32(b.dHp, P.n_split, (int64_t)Tc * d, dhf, s);
+        }));
+        if (!coll_rc) {
+          coll_rc = L.collective(KID_VP_REDUCE, (double)Tc * d * 4, [&] {
+            return group->all_reduce_sum(group->user, dhf, (int64_t)Tc * d, s);
+          });
+        }
+        chk(L(KID_TO_BF16, 0, (double)Tc * d * 6.0, [&] {
+          launch_f32_to_bf16(dhf, (int64_t)Tc * d, reinterpret_cast<uint16_t*>(dHc), s);
+        }));
+      }
       chk(L(KID_DW, zflops, 0, [&] {
         TcLaunch p{};
         p.kind = TcKind::DW; p.M = V; p.N = d; p.n_kb = (Tc + 63) / 64; p.n_split = 1;
@@ -364,6 +439,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     std::fprintf(stderr, "ckl: CUDA error: %s\n", cudaGetErrorString(err));
     return CKL_ERR_CUDA;
   }
+  if (coll_rc != 0) return CKL_ERR_COLLECTIVE;
   return CKL_OK;
 }
 
@@ -424,6 +500,7 @@ const char* ckl_status_str(ckl_status s) {
     case CKL_ERR_TIMEOUT: return "device pipeline wait timed out";
     case CKL_ERR_ALIGNMENT: return "pointer misaligned";
     case CKL_ERR_INTERNAL: return "internal consistency check failed";
+    case CKL_ERR_COLLECTIVE: return "a caller-supplied collective failed";
   }
   return "unknown status";
 }
@@ -539,6 +616,31 @@ ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t
   }
   return ckl_fwd_bwd(h, H_dev, W, idx_dev, logit_dev, mask_host ? mask_dev : nullptr, T, chunk,
                      loss, dH, dW, nullptr, nullptr, workspace, workspace_bytes, stream, loss_host);
+}
+
+ckl_status ckl_vp_workspace_bytes(ckl_handle h, int32_t world, int64_t T, int64_t chunk,
+                                  size_t* bytes) {
+  if (!h || !bytes || world < 1 || T < 0 || chunk < 1) return CKL_ERR_INVALID_ARG;
+  *bytes = plan(h, T, chunk, true, world).total;
+  return CKL_OK;
+}
+
+ckl_status ckl_fwd_bwd_vocab_parallel(ckl_handle h, const ckl_vocab_group* g, const void* H,
+                                      const void* W_shard, const int32_t* topk_idx,
+                                      const float* topk_logit, const uint8_t* mask, int64_t T,
+                                      int64_t chunk, float* loss, void* dH, float* dW_shard,
+                                      float* token_lse, float* token_loss, void* workspace,
+                                      size_t workspace_bytes, void* stream, float* loss_host) {
+  if (!h || !g || g->world < 1 || g->rank < 0 || g->rank >= g->world || !g->all_gather ||
+      !g->all_reduce_sum || g->v0 < 0 || g->V_total > INT32_MAX || g->v0 + h->V > g->V_total)
+    return CKL_ERR_INVALID_ARG;
+  if (h->dtype != CKL_BF16) return CKL_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ckl_status st = run(h, H, W_shard, topk_idx, topk_logit, mask, T, chunk, loss, dH, dW_shard,
+                      token_lse, token_loss, workspace, workspace_bytes, s, true, g);
+  if (st != CKL_OK || !loss_host) return st;
+  DeviceGuard guard(h->device);
+  return sync_and_read(h, s, loss, loss_host);
 }
 
 ckl_status ckl_sync_status(ckl_handle h, void* stream) {

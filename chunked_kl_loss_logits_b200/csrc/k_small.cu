@@ -32,21 +32,10 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Dot product of two 16-byte vectors of the input type.
+// Dot product of two 16-byte vectors of fp32 (the fp32 gather path).
 __device__ __forceinline__ float dot16(const uint4& a, const uint4& b, const float*) {
   return __uint_as_float(a.x) * __uint_as_float(b.x) + __uint_as_float(a.y) * __uint_as_float(b.y) +
          __uint_as_float(a.z) * __uint_as_float(b.z) + __uint_as_float(a.w) * __uint_as_float(b.w);
-}
-__device__ __forceinline__ float dot16(const uint4& a, const uint4& b, const __nv_bfloat16*) {
-  float s = lo_bf16(a.x) * lo_bf16(b.x);
-  s = fmaf(hi_bf16(a.x), hi_bf16(b.x), s);
-  s = fmaf(lo_bf16(a.y), lo_bf16(b.y), s);
-  s = fmaf(hi_bf16(a.y), hi_bf16(b.y), s);
-  s = fmaf(lo_bf16(a.z), lo_bf16(b.z), s);
-  s = fmaf(hi_bf16(a.z), hi_bf16(b.z), s);
-  s = fmaf(lo_bf16(a.w), lo_bf16(b.w), s);
-  s = fmaf(hi_bf16(a.w), hi_bf16(b.w), s);
-  return s;
 }
 
 constexpr int kGatherWarps = 4;
@@ -58,9 +47,12 @@ constexpr int kTeacherWarps = 8;
 //  3. ent = sum_k p_k log P_k
 //  4. the (id, p) pairs in ascending id order (ties in slot order), for the
 //     forward contraction's epilogue to pick z at the ids and form sum_k p_k z_k
+// Ids are checked against the full vocabulary V_all; the sorted ids are written
+// relative to v0, the first row of this caller's slice of the LM head (0 unless
+// the vocabulary is split over ranks), so ids outside the slice match no column.
 __global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
-    const int32_t* __restrict__ idx, const float* __restrict__ logit, int64_t t0, int Tc, int V,
-    int K, int k_bytes, float4* __restrict__ tok, float* __restrict__ Pk_out,
+    const int32_t* __restrict__ idx, const float* __restrict__ logit, int64_t t0, int Tc,
+    int V_all, int v0, int K, int k_bytes, float4* __restrict__ tok, float* __restrict__ Pk_out,
     int32_t* __restrict__ sid_out, float* __restrict__ sp_out, unsigned* status) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -95,7 +87,7 @@ __global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
   for (int k = lane; k < K; k += 32) {
     sP[k] = (live && se > 0.f) ? expf(sP[k] - mx) / se : 0.f;
     const int id = sId[k];
-    if (id < 0 || id >= V) atomicOr(status, (unsigned)ST_INDEX_RANGE);
+    if (id < 0 || id >= V_all) atomicOr(status, (unsigned)ST_INDEX_RANGE);
   }
   __syncwarp();
   float ent = 0.f, Msum = 0.f;
@@ -118,7 +110,7 @@ __global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
     if (p > 0.f) ent += p * logf(P);
     Msum += p;
     Pk_out[(int64_t)i * K + k] = first ? P : 0.f;
-    sid_out[(int64_t)i * K + rank] = id;
+    sid_out[(int64_t)i * K + rank] = id - v0;
     sp_out[(int64_t)i * K + rank] = p;
   }
   ent = warp_sum(ent);
@@ -259,15 +251,36 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
 
 constexpr int kCombTok = 32, kCombSplit = 32;
 
+// From a token's merged (max, sum) in log2 units and its cross term: lse,
+// l_t = ent - cross + M lse and the gradient multipliers.
+__device__ __forceinline__ void finish_token(int64_t t0, int i, float M2, float S, float cross,
+                                             const uint8_t* __restrict__ mask,
+                                             const float4* __restrict__ tok,
+                                             const Misc* __restrict__ misc, float4* __restrict__ cst,
+                                             float* __restrict__ lse_all,
+                                             float* __restrict__ ell_all) {
+  const float lse = (M2 + log2f(S)) * kLn2;
+  const float4 t4 = tok[i];
+  const float ell = t4.x - cross + t4.z * lse;
+  const int64_t t = t0 + i;
+  const float sc = (mask == nullptr || mask[t] != 0) ? misc->invN : 0.f;
+  cst[i] = make_float4(lse, sc * t4.z, sc, 0.f);
+  lse_all[t] = lse;
+  ell_all[t] = ell;
+}
+
 // Merge the per-vocabulary-tile (max, sum) partials into logsumexp(z_t), then
 // l_t = ent - cross + M lse and the gradient multipliers. A block covers 32
 // tokens; its 32 warps each merge every 32nd vocabulary tile (coalesced 256-byte
 // reads of 32 consecutive tokens), then one warp merges the 32 results.
+// With `stats` set (vocabulary split over ranks) it stops at this rank's
+// (max, sum, cross) per token; vp_merge_kernel finishes after the exchange.
 __global__ void __launch_bounds__(kCombTok * kCombSplit) combine_kernel(
     int64_t t0, int Tc, int n_vt, const uint8_t* __restrict__ mask,
     const float2* __restrict__ part, const float* __restrict__ xpart,
     const float4* __restrict__ tok, const Misc* __restrict__ misc,
-    float4* __restrict__ cst, float* __restrict__ lse_all, float* __restrict__ ell_all) {
+    float4* __restrict__ cst, float* __restrict__ lse_all, float* __restrict__ ell_all,
+    float4* __restrict__ stats) {
   __shared__ float sm[kCombSplit][kCombTok], ss[kCombSplit][kCombTok], sx[kCombSplit][kCombTok];
   const int tk = threadIdx.x % kCombTok, sp = threadIdx.x / kCombTok;
   const int i = blockIdx.x * kCombTok + tk;
@@ -299,15 +312,32 @@ __global__ void __launch_bounds__(kCombTok * kCombSplit) combine_kernel(
     if (sm[j][tk] > -INFINITY) S += ss[j][tk] * ex2_approx(sm[j][tk] - M2);
     X += sx[j][tk];
   }
-  const float lse = (M2 + log2f(S)) * kLn2;
-  const float4 t4 = tok[i];
-  const float cross = xpart ? X : t4.y;  // bf16: from the contraction's epilogue; fp32: gathered
-  const float ell = t4.x - cross + t4.z * lse;
-  const int64_t t = t0 + i;
-  const float sc = (mask == nullptr || mask[t] != 0) ? misc->invN : 0.f;
-  cst[i] = make_float4(lse, sc * t4.z, sc, 0.f);
-  lse_all[t] = lse;
-  ell_all[t] = ell;
+  const float cross = xpart ? X : tok[i].y;  // bf16: from the contraction's epilogue; fp32: gathered
+  if (stats) {
+    stats[i] = make_float4(M2, S, cross, 0.f);
+    return;
+  }
+  finish_token(t0, i, M2, S, cross, mask, tok, misc, cst, lse_all, ell_all);
+}
+
+// Vocabulary split over ranks: merge every rank's (max, sum, cross) of a token,
+// in rank order (stats_all is rank-major, world x Tc), so that every rank
+// computes the same lse and l_t bit for bit. One thread per token.
+__global__ void vp_merge_kernel(int64_t t0, int Tc, int world, const float4* __restrict__ stats_all,
+                                const uint8_t* __restrict__ mask, const float4* __restrict__ tok,
+                                const Misc* __restrict__ misc, float4* __restrict__ cst,
+                                float* __restrict__ lse_all, float* __restrict__ ell_all) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= Tc) return;
+  float M2 = -INFINITY;
+  for (int r = 0; r < world; ++r) M2 = fmaxf(M2, stats_all[(int64_t)r * Tc + i].x);
+  float S = 0.f, X = 0.f;
+  for (int r = 0; r < world; ++r) {
+    const float4 q = stats_all[(int64_t)r * Tc + i];
+    if (q.x > -INFINITY) S += q.y * ex2_approx(q.x - M2);
+    X += q.z;
+  }
+  finish_token(t0, i, M2, S, X, mask, tok, misc, cst, lse_all, ell_all);
 }
 
 // Stored-exp forward: the gradient buffer holds e = exp2(z log2e - m2_tile) in
@@ -343,9 +373,11 @@ __device__ __forceinline__ float load_g(const uint16_t* G, int64_t off) {
 
 // One thread per (token, slot) that holds the first occurrence of an id (P_k > 0):
 // overwrite: G[i][id] = gmul exp(z_k - lse) - s P_k;  else: G[i][id] -= s P_k.
+// Ids are taken relative to v0 (the slice's first row); ids outside [0, V) of
+// the slice belong to another rank and are skipped.
 template <typename Tg>
 __global__ void fixup_kernel(const int32_t* __restrict__ idx, int64_t t0, int Tc, int K, int V,
-                             int64_t ldG, const float4* __restrict__ cst,
+                             int v0, int64_t ldG, const float4* __restrict__ cst,
                              const float* __restrict__ zk, const float* __restrict__ Pk, Tg* G,
                              int overwrite) {
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -353,12 +385,37 @@ __global__ void fixup_kernel(const int32_t* __restrict__ idx, int64_t t0, int Tc
   const float P = Pk[e];
   if (!(P > 0.f)) return;
   const int64_t i = e / K;
-  const int id = idx[t0 * K + e];
+  const int id = idx[t0 * K + e] - v0;
   if (id < 0 || id >= V) return;
   const float4 c = cst[i];
   const int64_t off = i * ldG + id;
   const float g = overwrite ? c.y * expf(zk[e] - c.x) - c.z * P : load_g(G, off) - c.z * P;
   store_g(G, off, g);
+}
+
+// Sum of the split-K partials in fp32 (vocabulary split over ranks: the ranks'
+// sums are added by the exchange before the conversion to bf16).
+__global__ void dh_reduce_f32_kernel(const float* __restrict__ dHp, int n_split, int64_t n_elem,
+                                     float* __restrict__ out) {
+  const int64_t e4 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (e4 >= n_elem) return;
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < n_split; ++s) {
+    const float4 x = *reinterpret_cast<const float4*>(dHp + s * n_elem + e4);
+    a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+  }
+  *reinterpret_cast<float4*>(out + e4) = a;
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ in, int64_t n_elem,
+                                   uint16_t* __restrict__ out) {
+  const int64_t e4 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (e4 >= n_elem) return;
+  const float4 x = *reinterpret_cast<const float4*>(in + e4);
+  uint2 o;
+  o.x = pack_bf16x2(x.x, x.y);
+  o.y = pack_bf16x2(x.z, x.w);
+  *reinterpret_cast<uint2*>(out + e4) = o;
 }
 
 __global__ void dh_reduce_bf16_kernel(const float* __restrict__ dHp, int n_split, int64_t n_elem,
@@ -576,14 +633,14 @@ void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t 
   mask_count_kernel<<<1, kReduceThreads, 0, s>>>(mask, T, misc);
 }
 
-void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V, int K,
-                    const ChunkBufs& b, unsigned* status, cudaStream_t s) {
+void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V_all, int v0,
+                    int K, const ChunkBufs& b, unsigned* status, cudaStream_t s) {
   const int k_bytes = (K * 4 + 15) & ~15;
   const size_t smem = (size_t)kTeacherWarps * 2 * k_bytes;
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(teacher_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   teacher_kernel<<<blocks_for(Tc, kTeacherWarps), kTeacherWarps * 32, smem, s>>>(
-      idx, logit, t0, Tc, V, K, k_bytes, b.tok, b.Pk, b.sid, b.sp, status);
+      idx, logit, t0, Tc, V_all, v0, K, k_bytes, b.tok, b.Pk, b.sid, b.sp, status);
 }
 
 template <typename Tin>
@@ -605,9 +662,15 @@ template void launch_gather<float>(const float*, const float*, const int32_t*, c
                                    cudaStream_t);
 
 void launch_combine(int64_t t0, int Tc, int n_vt, const uint8_t* mask, const ChunkBufs& b,
-                    float* lse_all, float* ell_all, cudaStream_t s) {
+                    float* lse_all, float* ell_all, float4* stats, cudaStream_t s) {
   combine_kernel<<<blocks_for(Tc, kCombTok), kCombTok * kCombSplit, 0, s>>>(
-      t0, Tc, n_vt, mask, b.part, b.xpart, b.tok, b.misc, b.cst, lse_all, ell_all);
+      t0, Tc, n_vt, mask, b.part, b.xpart, b.tok, b.misc, b.cst, lse_all, ell_all, stats);
+}
+
+void launch_vp_merge(int64_t t0, int Tc, int world, const float4* stats_all, const uint8_t* mask,
+                     const ChunkBufs& b, float* lse_all, float* ell_all, cudaStream_t s) {
+  vp_merge_kernel<<<blocks_for(Tc, 128), 128, 0, s>>>(t0, Tc, world, stats_all, mask, b.tok,
+                                                      b.misc, b.cst, lse_all, ell_all);
 }
 
 void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s) {
@@ -616,19 +679,28 @@ void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b,
 }
 
 template <typename Tg>
-void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int64_t ldG,
+void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int v0, int64_t ldG,
                   const ChunkBufs& b, bool overwrite, cudaStream_t s) {
   fixup_kernel<Tg><<<blocks_for((int64_t)Tc * K, 256), 256, 0, s>>>(
-      idx, t0, Tc, K, V, ldG, b.cst, b.zk, b.Pk, static_cast<Tg*>(b.G), overwrite ? 1 : 0);
+      idx, t0, Tc, K, V, v0, ldG, b.cst, b.zk, b.Pk, static_cast<Tg*>(b.G), overwrite ? 1 : 0);
 }
-template void launch_fixup<float>(const int32_t*, int64_t, int, int, int, int64_t,
+template void launch_fixup<float>(const int32_t*, int64_t, int, int, int, int, int64_t,
                                   const ChunkBufs&, bool, cudaStream_t);
-template void launch_fixup<uint16_t>(const int32_t*, int64_t, int, int, int, int64_t,
+template void launch_fixup<uint16_t>(const int32_t*, int64_t, int, int, int, int, int64_t,
                                      const ChunkBufs&, bool, cudaStream_t);
 
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
                            cudaStream_t s) {
   dh_reduce_bf16_kernel<<<blocks_for(n_elem / 8, 256), 256, 0, s>>>(dHp, n_split, n_elem, dH);
+}
+
+void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out,
+                          cudaStream_t s) {
+  dh_reduce_f32_kernel<<<blocks_for(n_elem / 4, 256), 256, 0, s>>>(dHp, n_split, n_elem, out);
+}
+
+void launch_f32_to_bf16(const float* in, int64_t n_elem, uint16_t* out, cudaStream_t s) {
+  f32_to_bf16_kernel<<<blocks_for(n_elem / 4, 256), 256, 0, s>>>(in, n_elem, out);
 }
 
 void launch_topk_threshold(const float2* tbest, int n_vt, int rows, int K, float2* theta,

@@ -42,6 +42,8 @@
 // Operand layouts: H, W and G are read K-major for LSE/GRAD/DH-A; W (DH-B), G
 // (DW-A) and H (DW-B) are read MN-major, so no operand is ever transposed in
 // memory. No load uses cluster multicast. Every wait is bounded (common.cuh).
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -533,7 +535,9 @@ cudaError_t launch_kind(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // As many pairs as can be resident at once (one CTA per SM), at most one per tile.
-  static int max_pairs = 0;
+  // Cached per kind; concurrent first calls compute the same value.
+  static std::atomic<int> cached_pairs{0};
+  int max_pairs = cached_pairs.load(std::memory_order_relaxed);
   if (max_pairs == 0) {
     cfg.gridDim = dim3(2 * p.num_sms, 1, 1);
     int clusters = 0;
@@ -541,6 +545,7 @@ cudaError_t launch_kind(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
         clusters < 1)
       clusters = p.num_sms / 2;
     max_pairs = clusters;
+    cached_pairs.store(max_pairs, std::memory_order_relaxed);
   }
   const int pairs = n_tiles < max_pairs ? n_tiles : max_pairs;
   cfg.gridDim = dim3(2 * pairs, 1, 1);

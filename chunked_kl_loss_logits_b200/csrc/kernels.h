@@ -38,24 +38,34 @@ struct Misc {
 void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t s);
 // bf16: teacher softmax, merged P, entropy term and each token's ids sorted with
 // their probabilities (the forward contraction picks the student logits there).
-void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V, int K,
-                    const ChunkBufs& b, unsigned* status, cudaStream_t s);
+// Ids are checked against V_all and written relative to v0 (vocabulary split
+// over ranks: this rank holds rows [v0, v0 + V) of W; otherwise v0 = 0, V_all = V).
+void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V_all, int v0,
+                    int K, const ChunkBufs& b, unsigned* status, cudaStream_t s);
 // fp32: as launch_teacher, plus the student logits at the ids by dot products.
 template <typename Tin>
 void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* logit, int64_t t0,
                    int Tc, int d, int V, int K, const ChunkBufs& b, unsigned* status,
                    cudaStream_t s);
+// stats != nullptr: write this rank's per-token (max2, sum, cross, 0) and stop.
 void launch_combine(int64_t t0, int Tc, int n_vt, const uint8_t* mask, const ChunkBufs& b,
-                    float* lse_all, float* ell_all, cudaStream_t s);
+                    float* lse_all, float* ell_all, float4* stats, cudaStream_t s);
+// Merge world x Tc gathered stats (rank-major) into lse, l_t and the multipliers.
+void launch_vp_merge(int64_t t0, int Tc, int world, const float4* stats_all, const uint8_t* mask,
+                     const ChunkBufs& b, float* lse_all, float* ell_all, cudaStream_t s);
 // G at the cached ids. overwrite: G = gmul exp(z_k - lse) - s P_k (the gradient
 // contraction wrote gmul exp(z - lse) there); otherwise G -= s P_k in place.
 template <typename Tg>
-void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int64_t ldG,
+void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int v0, int64_t ldG,
                   const ChunkBufs& b, bool overwrite, cudaStream_t s);
 // Stored-exp forward: G[i][v] = e[i][v] * gmul_i * exp2(m2[tile(v)][i] - lse_i log2 e), in place.
 void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s);
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
                            cudaStream_t s);
+// n_elem % 4 == 0
+void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out,
+                          cudaStream_t s);
+void launch_f32_to_bf16(const float* in, int64_t n_elem, uint16_t* out, cudaStream_t s);
 // Teacher top-K cache: per row, the threshold = the K-th best of the n_vt tile
 // bests (logit descending, id ascending), or "take everything" when n_vt <= K.
 void launch_topk_threshold(const float2* tbest, int n_vt, int rows, int K, float2* theta,

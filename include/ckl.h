@@ -62,7 +62,8 @@ typedef enum {
   CKL_ERR_CUDA = 5,         /* a CUDA runtime call failed (no device, launch failure, ...) */
   CKL_ERR_TIMEOUT = 6,      /* device: a pipeline wait exceeded its bound; the kernel gave up */
   CKL_ERR_ALIGNMENT = 7,    /* a pointer is not aligned as stated above */
-  CKL_ERR_INTERNAL = 8      /* device: an internal consistency check failed */
+  CKL_ERR_INTERNAL = 8,     /* device: an internal consistency check failed */
+  CKL_ERR_COLLECTIVE = 9    /* a caller-supplied collective returned nonzero */
 } ckl_status;
 
 typedef enum { CKL_F32 = 0, CKL_BF16 = 1 } ckl_dtype;
@@ -168,6 +169,57 @@ ckl_status ckl_topk_workspace_bytes(ckl_handle h, int64_t T, int64_t chunk, size
 ckl_status ckl_topk_cache(ckl_handle h, const void* H, const void* W, int64_t T, int64_t chunk,
                           int32_t* topk_idx, float* topk_logit, void* workspace,
                           size_t workspace_bytes, void* stream, int wait);
+
+/* ---- Vocabulary-parallel loss (tensor parallelism over the LM head) ----
+ *
+ * The benchmark on the page "Chunked KL loss, running Knowledge Distillation
+ * locally in less <6GB VRAM" runs its losses tensor-parallel (options table,
+ * `--tp`) without describing the split; this is the split of the LM head by
+ * vocabulary rows. The ranks of a group hold the same tokens (H, ids, logits,
+ * mask) and disjoint, contiguous row ranges of W: this rank holds rows
+ * [v0, v0 + V) of the full V_total x d head, V being its handle's V. Per chunk,
+ * each rank reduces its own logits to per-token (max, sum of exp, sum of p z at
+ * the cached ids inside its rows); the group all-gathers those triples and every
+ * rank merges them in rank order, so lse, the per-token losses and the loss are
+ * the same on every rank, bit for bit. dH = sum over ranks of G_r W_r is summed
+ * in fp32 by an all-reduce per chunk; dW_r = G_r^T H stays on its rank.
+ * The library calls no collective library itself: the caller supplies the two
+ * collectives (NCCL, torch.distributed, MPI, ...). Each must be ordered on the
+ * `stream` it is given (enqueued there, or complete when it returns) and return
+ * 0 on success. Every rank makes the same sequence of collective calls, one
+ * all-gather per chunk and one all-reduce per chunk (T = 0: none). After a
+ * kernel failure the remaining collectives are still made (the group stays
+ * matched) and the call returns CKL_ERR_CUDA; after a collective returns
+ * nonzero no further collective is called and the call returns
+ * CKL_ERR_COLLECTIVE. Argument errors are returned before any collective.
+ * bf16 handles only; world = 1 gives the result of ckl_fwd_bwd. */
+typedef int (*ckl_all_gather_fn)(void* user, const float* send, float* recv, int64_t count,
+                                 void* stream);  /* recv: world x count floats, rank-major */
+typedef int (*ckl_all_reduce_sum_fn)(void* user, float* buf, int64_t count,
+                                     void* stream);  /* in place, element-wise sum */
+typedef struct {
+  int32_t world;   /* ranks in the group (>= 1) */
+  int32_t rank;    /* this rank (0 <= rank < world) */
+  int64_t V_total; /* full vocabulary size: ids are checked against it */
+  int64_t v0;      /* first vocabulary row held by this rank (v0 + V <= V_total) */
+  ckl_all_gather_fn all_gather;
+  ckl_all_reduce_sum_fn all_reduce_sum;
+  void* user;      /* passed back to both functions */
+} ckl_vocab_group;
+
+/* Workspace of ckl_fwd_bwd_vocab_parallel: ckl_workspace_bytes plus
+ * chunk * (16 (world + 1) + 4 d) bytes for the exchanged statistics and dH. */
+ckl_status ckl_vp_workspace_bytes(ckl_handle h, int32_t world, int64_t T, int64_t chunk,
+                                  size_t* bytes);
+/* As ckl_fwd_bwd with W_shard (V x d, this rank's rows) and dW_shard (V x d
+ * fp32); H, ids, logits, mask, loss, dH, token_lse and token_loss as there
+ * (full-vocabulary values, identical on every rank). */
+ckl_status ckl_fwd_bwd_vocab_parallel(ckl_handle h, const ckl_vocab_group* group, const void* H,
+                                      const void* W_shard, const int32_t* topk_idx,
+                                      const float* topk_logit, const uint8_t* mask, int64_t T,
+                                      int64_t chunk, float* loss, void* dH, float* dW_shard,
+                                      float* token_lse, float* token_loss, void* workspace,
+                                      size_t workspace_bytes, void* stream, float* loss_host);
 
 /* Wait for `stream` and return the device-detected status of the calls enqueued
  * on it since the last synchronising call (clears it). */

@@ -26,7 +26,7 @@ def test_exports_every_declared_function(L):
 
 
 def test_status_strings(L):
-    for code in range(9):
+    for code in range(10):
         s = L.ckl_status_str(code)
         assert s and s != b"unknown status"
     assert L.ckl_status_str(99) == b"unknown status"
@@ -67,3 +67,6 @@ def test_null_handle_calls(L):
     assert L.ckl_launch_count(None) == -1
     assert L.ckl_destroy(None) == 0
     assert L.ckl_profile_enable(None, 1, 16) == 1
+    assert L.ckl_vp_workspace_bytes(None, 2, 10, 4, ctypes.byref(n)) == 1
+    assert L.ckl_fwd_bwd_vocab_parallel(None, None, *([None] * 5), 10, 4, *([None] * 6), 0, None,
+                                        None) == 1

@@ -61,6 +61,8 @@ def test_tiny_f32_workload_full():
     (50, 64, 100, 7, 32),         # V smaller than one vocabulary tile, K % 4 != 0
     (129, 2880, 3001, 100, 129),  # the headline hidden size and K, odd V
     (384, 192, 2048, 32, 384),    # exact multiples everywhere
+    (600, 384, 5000, 20, 600),    # narrow last hidden-size tile (128 of 256 columns), 3 row tiles
+    (300, 296, 2500, 8, 300),     # narrow last hidden-size tile with 40 valid columns
 ])
 @pytest.mark.parametrize("recompute", [False, True], ids=["stored", "recompute"])
 def test_bf16_ragged_shapes(T, d, V, K, chunk, recompute):

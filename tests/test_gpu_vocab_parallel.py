@@ -1,0 +1,185 @@
+"""Vocabulary-parallel loss through the C ABI, against the fp64 oracle.
+
+The ranks of a group run as threads of this process on one GPU, each with its
+own handle and stream; the group's collectives meet on the host (each rank's
+stream is synchronised before its buffer is shared and after the result is
+written back), so no kernel ever waits for another. Checked: loss, dH, lse and
+per-token loss identical bit for bit on every rank; loss, lse, dH and the
+concatenated dW shards equal to the oracle within the bf16 tolerances; a group
+of one equal to the single-rank call; a failing collective reported as
+CKL_ERR_COLLECTIVE with no further collective called.
+"""
+import threading
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_kl_loss_logits_b200 import ckl
+from chunked_kl_loss_logits_b200.workloads import small_case
+
+pytestmark = pytest.mark.gpu
+
+
+class ThreadGroup:
+    """`world` ranks as threads; collectives exchange device tensors through the host side."""
+
+    def __init__(self, world):
+        self.world = world
+        self.barrier = threading.Barrier(world, timeout=120)
+        self.slots = [None] * world
+        self.calls = [[] for _ in range(world)]
+
+    def member(self, rank, V_total, v0):
+        def all_gather(send, recv):
+            self.calls[rank].append(("gather", send.numel()))
+            torch.cuda.current_stream().synchronize()
+            self.slots[rank] = send.clone()
+            torch.cuda.current_stream().synchronize()
+            self.barrier.wait()
+            n = send.numel()
+            for r in range(self.world):
+                recv[r * n:(r + 1) * n].copy_(self.slots[r])
+            torch.cuda.current_stream().synchronize()
+            self.barrier.wait()
+
+        def all_reduce_sum(buf):
+            self.calls[rank].append(("reduce", buf.numel()))
+            torch.cuda.current_stream().synchronize()
+            self.slots[rank] = buf.clone()
+            torch.cuda.current_stream().synchronize()
+            self.barrier.wait()
+            acc = self.slots[0].clone()
+            for r in range(1, self.world):  # rank order: the same sum on every rank
+                acc += self.slots[r]
+            buf.copy_(acc)
+            torch.cuda.current_stream().synchronize()
+            self.barrier.wait()
+
+        return ckl.VocabGroup(self.world, rank, V_total, v0, all_gather, all_reduce_sum)
+
+
+def run_group(x, world, chunk, shards=None):
+    T, d = x["H"].shape
+    V = x["W"].shape[0]
+    K = x["idx"].shape[1]
+    shards = shards or ckl.vocab_shards(V, world)
+    dev = torch.device("cuda", 0)
+    H = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
+    W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+    idx = torch.from_numpy(x["idx"]).to(dev)
+    lg = torch.from_numpy(x["logit"]).to(dev)
+    mask = torch.from_numpy(x["mask"]).to(dev) if x.get("mask") is not None else None
+    torch.cuda.synchronize(dev)  # inputs ready before the ranks' streams read them
+    tg = ThreadGroup(world)
+    out, errs = [None] * world, []
+
+    def rank_main(r):
+        try:
+            torch.cuda.set_device(dev)
+            v0, n = shards[r]
+            h = ckl.ChunkedKL(n, d, K, max_chunk=chunk, device=dev)
+            s = torch.cuda.Stream(dev)
+            with torch.cuda.stream(s):
+                W_r = W[v0:v0 + n].contiguous()
+                s.synchronize()
+                res = h.fwd_bwd_vocab_parallel(tg.member(r, V, v0), H, W_r, idx, lg, mask,
+                                               chunk=chunk, token_stats=True)
+                s.synchronize()
+            out[r] = [t.cpu() for t in res]
+            h.close()
+        except Exception as e:  # surfaced by the test
+            errs.append(e)
+            tg.barrier.abort()
+
+    th = [threading.Thread(target=rank_main, args=(r,)) for r in range(world)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join(300)
+    assert not errs, errs
+    return out, tg, shards
+
+
+def check_against_oracle(x, out, shards):
+    r = oracle.fwd_bwd(x["H"], x["W"], x["idx"], x["logit"], x.get("mask"))
+    loss, dH, _, lse, ell = out[0]
+    for o in out[1:]:  # identical on every rank
+        for a, b in ((loss, o[0]), (dH, o[1]), (lse, o[3]), (ell, o[4])):
+            assert torch.equal(a, b)
+    assert abs(float(loss) - r["loss"]) <= 1e-3 * max(1.0, abs(r["loss"]))
+    np.testing.assert_allclose(lse.numpy(), r["lse"], rtol=0, atol=2e-6 * np.abs(r["lse"]).max() + 1e-5)
+    scale = np.abs(r["dH"]).max()
+    assert np.abs(dH.float().numpy() - r["dH"]).max() <= 1e-2 * scale
+    dW = torch.cat([o[2] for o in out]).numpy()
+    assert dW.shape == r["dW"].shape
+    assert np.abs(dW - r["dW"]).max() <= 1e-2 * np.abs(r["dW"]).max()
+
+
+@pytest.mark.parametrize("world,T,d,V,K,chunk", [
+    (2, 300, 128, 3000, 16, 128),    # two shards, ragged chunks
+    (3, 257, 64, 1000, 12, 100),     # uneven shards (512, 256, 232 rows)
+    (4, 129, 2880, 3001, 100, 129),  # the headline hidden size and K
+])
+def test_group_matches_oracle(world, T, d, V, K, chunk):
+    x = small_case(T, d, V, K, seed=world * 100 + T, dtype="bf16", teacher_var=3.0, ids="zipf")
+    out, tg, shards = run_group(x, world, chunk)
+    check_against_oracle(x, out, shards)
+    n_chunks = (T + chunk - 1) // chunk
+    for calls in tg.calls:  # one gather and one reduce per chunk, the same on every rank
+        assert [c[0] for c in calls] == ["gather", "reduce"] * n_chunks
+    assert tg.calls[0] == tg.calls[-1]
+
+
+def test_group_with_mask():
+    x = small_case(300, 64, 1500, 16, seed=31, dtype="bf16", packing=True)
+    out, _, shards = run_group(x, 2, 128)
+    check_against_oracle(x, out, shards)
+
+
+def test_group_of_one_equals_single_rank_call():
+    x = small_case(200, 128, 2000, 16, seed=32, dtype="bf16")
+    out, _, _ = run_group(x, 1, 64)
+    dev = torch.device("cuda", 0)
+    h = ckl.ChunkedKL(2000, 128, 16, max_chunk=64, device=dev)
+    H = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
+    W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+    loss, dH, dW, lse, ell = h.fwd_bwd(H, W, torch.from_numpy(x["idx"]).to(dev),
+                                       torch.from_numpy(x["logit"]).to(dev), chunk=64,
+                                       token_stats=True)
+    assert torch.equal(dH.cpu(), out[0][1]) and torch.equal(dW.cpu(), out[0][2])
+    torch.testing.assert_close(lse.cpu(), out[0][3], rtol=1e-6, atol=1e-6)
+    torch.testing.assert_close(loss.cpu(), out[0][0], rtol=1e-6, atol=1e-7)
+
+
+def test_failing_collective_is_reported():
+    x = small_case(100, 64, 500, 8, seed=33, dtype="bf16")
+    dev = torch.device("cuda", 0)
+    calls = []
+
+    def bad_gather(send, recv):
+        calls.append("gather")
+        raise RuntimeError("peer lost")
+
+    def reduce(buf):
+        calls.append("reduce")
+
+    g = ckl.VocabGroup(1, 0, 500, 0, bad_gather, reduce)
+    h = ckl.ChunkedKL(500, 64, 8, max_chunk=32, device=dev)
+    H = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
+    W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+    with pytest.raises(ckl.CKLError) as ei:
+        h.fwd_bwd_vocab_parallel(g, H, W, torch.from_numpy(x["idx"]).to(dev),
+                                 torch.from_numpy(x["logit"]).to(dev), chunk=32)
+    assert ei.value.code == 9 and isinstance(ei.value.__cause__, RuntimeError)
+    assert calls == ["gather"]  # no collective after the failed one
+    torch.cuda.synchronize()
+
+
+def test_ids_outside_the_full_vocabulary_are_reported():
+    x = small_case(64, 64, 600, 8, seed=34, dtype="bf16")
+    x["idx"][3, 2] = 600
+    with pytest.raises(AssertionError) as ei:
+        run_group(x, 2, 32)
+    assert "top-K index out of range" in str(ei.value)

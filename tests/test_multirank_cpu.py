@@ -38,7 +38,7 @@ def _worker(rank, world, port, times, out):
 def test_max_over_ranks_and_job_rate(times):
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     ctx = mp.get_context("spawn")
     procs = [ctx.Process(target=_worker, args=(r, world, port, times, out)) for r in range(world)]
