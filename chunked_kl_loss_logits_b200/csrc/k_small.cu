@@ -342,24 +342,36 @@ __global__ void vp_merge_kernel(int64_t t0, int Tc, int world, const float4* __r
 
 // Stored-exp forward: the gradient buffer holds e = exp2(z log2e - m2_tile) in
 // bf16; turn it into G = gmul exp(z - lse) = e * gmul * exp2(m2_tile - lse log2e)
-// in place. A thread handles 8 consecutive columns of one row.
-__global__ void scale_e_kernel(uint16_t* __restrict__ G, int64_t ldG, int Tc, int V,
-                               const float2* __restrict__ part, const float4* __restrict__ cst) {
+// in place. Block (row i = blockIdx.x, 512 16-byte groups from blockIdx.y * 512):
+// each thread loads two 16-byte groups 256 apart before scaling either, so two
+// loads per thread are in flight.
+__global__ void __launch_bounds__(256) scale_e_kernel(uint16_t* __restrict__ G, int64_t ldG,
+                                                      int Tc, int V,
+                                                      const float2* __restrict__ part,
+                                                      const float4* __restrict__ cst) {
   const int n8 = (V + 7) / 8;
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= (int64_t)Tc * n8) return;
-  const int i = (int)(e / n8);
-  const int c8 = (int)(e - (int64_t)i * n8) * 8;
+  const int i = blockIdx.x;
+  const int q0 = blockIdx.y * 512 + threadIdx.x, q1 = q0 + 256;
   const float4 c = cst[i];
-  const float m2 = part[(int64_t)(c8 >> 8) * Tc + i].x;
-  const float f = c.y * ex2_approx(m2 - c.x * 1.4426950408889634f);
-  uint4* p = reinterpret_cast<uint4*>(G + (int64_t)i * ldG + c8);
-  uint4 x = *p;
-  x.x = pack_bf16x2(lo_bf16(x.x) * f, hi_bf16(x.x) * f);
-  x.y = pack_bf16x2(lo_bf16(x.y) * f, hi_bf16(x.y) * f);
-  x.z = pack_bf16x2(lo_bf16(x.z) * f, hi_bf16(x.z) * f);
-  x.w = pack_bf16x2(lo_bf16(x.w) * f, hi_bf16(x.w) * f);
-  *p = x;
+  const float l2 = c.x * 1.4426950408889634f;
+  uint16_t* row = G + (int64_t)i * ldG;
+  uint4 x[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  const int q[2] = {q0, q1};
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+    if (q[u] < n8) x[u] = *reinterpret_cast<const uint4*>(row + (int64_t)q[u] * 8);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    if (q[u] >= n8) continue;
+    // 32 groups of 8 columns per 256-column vocabulary tile
+    const float f = c.y * ex2_approx(part[(int64_t)(q[u] >> 5) * Tc + i].x - l2);
+    uint4 y = x[u];
+    y.x = pack_bf16x2(lo_bf16(y.x) * f, hi_bf16(y.x) * f);
+    y.y = pack_bf16x2(lo_bf16(y.y) * f, hi_bf16(y.y) * f);
+    y.z = pack_bf16x2(lo_bf16(y.z) * f, hi_bf16(y.z) * f);
+    y.w = pack_bf16x2(lo_bf16(y.w) * f, hi_bf16(y.w) * f);
+    *reinterpret_cast<uint4*>(row + (int64_t)q[u] * 8) = y;
+  }
 }
 
 __device__ __forceinline__ void store_g(float* G, int64_t off, float v) { G[off] = v; }
@@ -674,8 +686,8 @@ void launch_vp_merge(int64_t t0, int Tc, int world, const float4* stats_all, con
 }
 
 void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s) {
-  scale_e_kernel<<<blocks_for((int64_t)Tc * ((V + 7) / 8), 256), 256, 0, s>>>(G, ldG, Tc, V,
-                                                                            b.part, b.cst);
+  const dim3 grid((unsigned)Tc, (unsigned)(((V + 7) / 8 + 511) / 512));
+  scale_e_kernel<<<grid, 256, 0, s>>>(G, ldG, Tc, V, b.part, b.cst);
 }
 
 template <typename Tg>

@@ -183,3 +183,77 @@ def test_ids_outside_the_full_vocabulary_are_reported():
     with pytest.raises(AssertionError) as ei:
         run_group(x, 2, 32)
     assert "top-K index out of range" in str(ei.value)
+
+
+def test_group_in_recompute_mode():
+    # the backward forms the logits again from the merged lse
+    x = small_case(260, 64, 2000, 10, seed=35, dtype="bf16", teacher_var=3.0, ids="zipf")
+    orig = ckl.ChunkedKL.fwd_bwd_vocab_parallel
+
+    def with_recompute(self, *a, **k):
+        self.set_recompute(True)
+        return orig(self, *a, **k)
+
+    ckl.ChunkedKL.fwd_bwd_vocab_parallel = with_recompute
+    try:
+        out, _, shards = run_group(x, 2, 100)
+    finally:
+        ckl.ChunkedKL.fwd_bwd_vocab_parallel = orig
+    check_against_oracle(x, out, shards)
+
+
+def test_group_ragged_k_and_chunks():
+    x = small_case(77, 136, 1301, 7, seed=36, dtype="bf16")  # K % 4 != 0, d % 64 != 0
+    out, _, shards = run_group(x, 3, 32)
+    check_against_oracle(x, out, shards)
+
+
+@pytest.mark.parametrize("bad", ["rank", "v0", "world", "callback", "f32"])
+def test_group_arguments_are_checked(bad):
+    import ctypes
+    dev = torch.device("cuda", 0)
+    V, d, K = 512, 64, 8
+    dt = torch.float32 if bad == "f32" else torch.bfloat16
+    h = ckl.ChunkedKL(V, d, K, dtype=dt, max_chunk=32, device=dev)
+    calls = []
+    g = ckl.VocabGroup(2, 0, 1024, 0, lambda s, r: calls.append(1), lambda b: calls.append(2))
+    if bad == "rank":
+        g.rank = 2
+    elif bad == "v0":
+        g.v0 = 600  # 600 + 512 > 1024
+    elif bad == "world":
+        g.world = 0
+    H = torch.zeros((16, d), dtype=dt, device=dev)
+    W = torch.zeros((V, d), dtype=dt, device=dev)
+    idx = torch.zeros((16, K), dtype=torch.int32, device=dev)
+    lg = torch.zeros((16, K), dtype=torch.float32, device=dev)
+    if bad == "callback":
+        c, keep = g._c(dev)
+        c.all_gather = ckl._GatherFn()  # null function pointer
+        n = ctypes.c_size_t()
+        ckl.lib().ckl_vp_workspace_bytes(h._h, 2, 16, 32, ctypes.byref(n))
+        ws = torch.empty(n.value, dtype=torch.uint8, device=dev)
+        out = [torch.empty((), device=dev), torch.empty_like(H), torch.empty((V, d), device=dev)]
+        code = ckl.lib().ckl_fwd_bwd_vocab_parallel(
+            h._h, ctypes.byref(c), ckl._ptr(H), ckl._ptr(W), ckl._ptr(idx), ckl._ptr(lg), None, 16,
+            32, ckl._ptr(out[0]), ckl._ptr(out[1]), ckl._ptr(out[2]), None, None, ckl._ptr(ws),
+            ws.numel(), None, None)
+        assert code == 1
+    else:
+        with pytest.raises(ckl.CKLError) as ei:
+            h.fwd_bwd_vocab_parallel(g, H, W, idx, lg, chunk=32)
+        assert ei.value.code == (2 if bad == "f32" else 1)
+    assert calls == []  # argument errors come before any collective
+
+
+def test_empty_input_makes_no_collective_call():
+    dev = torch.device("cuda", 0)
+    calls = []
+    g = ckl.VocabGroup(1, 0, 512, 0, lambda s, r: calls.append(1), lambda b: calls.append(2))
+    h = ckl.ChunkedKL(512, 64, 8, max_chunk=32, device=dev)
+    H = torch.zeros((0, 64), dtype=torch.bfloat16, device=dev)
+    W = torch.randn((512, 64), device=dev).to(torch.bfloat16)
+    loss, dH, dW = h.fwd_bwd_vocab_parallel(g, H, W, torch.zeros((0, 8), dtype=torch.int32,
+                                                                   device=dev),
+                                            torch.zeros((0, 8), device=dev), chunk=32)
+    assert calls == [] and float(loss) == 0.0 and torch.count_nonzero(dW) == 0
