@@ -256,9 +256,13 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     sampler.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # one event between consecutive steps as well (recorded on the stream, no sync)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(max(0, args.steps - 1))]
     e0.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
         step()
+        if i < args.steps - 1:
+            ev[i].record(stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -266,6 +270,8 @@ def run_ours(args, w, rank, world, local_rank):
     launches = h.launch_count() - n_launch0
     h.sync_status()
     ms_max = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    marks = [e0] + ev + [e1]
+    per_step = [a.elapsed_time(b) for a, b in zip(marks, marks[1:])]
     stats = h.profile_collect()
     h.profile_enable(False, 0)
     peak_mem = torch.cuda.max_memory_allocated(dev) / 2**30
@@ -329,10 +335,12 @@ def run_ours(args, w, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "ms_per_step_median_rank0": statistics.median(per_step),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
         "config": {"workload": w.name, "T": w.T, "d": w.d, "V": w.V, "K": w.K, "chunk": chunk,
+                   "valid_tokens": int(w.T if x["mask"] is None else int(x["mask"].astype(bool).sum())),
                    "backward": ("recompute logits" if args.recompute or w.dtype != "bf16"
                                 else "stored exp(z), bf16"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
