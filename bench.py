@@ -543,6 +543,74 @@ def run_compare(args, w):
         del H0, W0, idx, lg
 
 
+def run_graph_compare(args, w):
+    """One workload's step, eager vs captured once in a CUDA graph and replayed.
+
+    Prints one JSON line (kind "graph"): mean ms per step of each over the same
+    number of timed steps (CUDA events, after warm-up). The graph holds the
+    call's launches, memsets and copies; replaying it removes the host launch
+    cost, which matters when the kernels are short (small workloads).
+    """
+    import torch
+
+    from chunked_kl_loss_logits_b200 import ckl
+    from chunked_kl_loss_logits_b200.workloads import make_inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    chunk = args.chunk or w.chunk
+    x = make_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    H = torch.from_numpy(x["H"]).to(dev).to(tdt)
+    W = torch.from_numpy(x["W"]).to(dev).to(tdt)
+    idx = torch.from_numpy(x["idx"]).to(dev)
+    logit = torch.from_numpy(x["logit"]).to(dev)
+    mask = None if x["mask"] is None else torch.from_numpy(x["mask"]).to(dev)
+    h = ckl.ChunkedKL(w.V, w.d, w.K, dtype=tdt, max_chunk=chunk, device=dev)
+    ws = h.workspace(w.T, chunk)
+    out = (torch.empty((), dtype=torch.float32, device=dev), torch.empty_like(H),
+           torch.empty((w.V, w.d), dtype=torch.float32, device=dev))
+
+    def step():
+        h.fwd_bwd(H, W, idx, logit, mask, chunk=chunk, out=out, workspace=ws, sync=False)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _ in range(max(3, args.warmup)):
+            step()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    n0 = h.launch_count()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    per_step = h.launch_count() - n0
+    h.sync_status()
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    eager = timed(step)
+    graph = timed(g.replay)
+    h.sync_status()
+    print(json.dumps({"kind": "graph", "workload": w.name, "T": w.T, "chunk": chunk,
+                      "steps": args.steps, "launches_per_step": per_step,
+                      "eager_ms": eager, "graph_ms": graph,
+                      "tokens_per_s_eager": w.T / (eager / 1e3),
+                      "tokens_per_s_graph": w.T / (graph / 1e3)}), flush=True)
+    del g
+    h.close()
+
+
 def run_topk_cache(args, w):
     """Teacher top-K cache builder on one workload's shape: tokens/s of one cache pass.
 
@@ -610,6 +678,8 @@ def main():
     ap.add_argument("--compare-tokens", type=lambda v: [int(t) for t in v.split(",")],
                     default=[4096, 8192, 16384, 32768])
     ap.add_argument("--compare-steps", type=int, default=3)
+    ap.add_argument("--graph-compare", action="store_true",
+                    help="the workload's step eager vs replayed from a CUDA graph (extra JSON line)")
     ap.add_argument("--topk-cache", action="store_true",
                     help="time the teacher top-K cache builder on the workload's shape instead")
     ap.add_argument("--recompute", action="store_true",
@@ -634,6 +704,9 @@ def main():
         return
     if args.topk_cache:
         run_topk_cache(args, w)
+        return
+    if args.graph_compare:
+        run_graph_compare(args, w)
         return
     if args.compare:
         run_compare(args, w)

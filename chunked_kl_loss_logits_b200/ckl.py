@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
                                    ctypes.c_int),
         "ckl_fwd_bwd_vocab_parallel": ([_P, ctypes.POINTER(_VocabGroupC), _P, _P, _P, _P, _P, _I64,
                                         _I64, _P, _P, _P, _P, _P, _P, _SZ, _P, _P], ctypes.c_int),
+        "ckl_forward_vocab_parallel": ([_P, ctypes.POINTER(_VocabGroupC), _P, _P, _P, _P, _P, _I64,
+                                        _I64, _P, _P, _P, _P, _SZ, _P, _P], ctypes.c_int),
         "ckl_profile_enable": ([_P, ctypes.c_int, ctypes.c_int], ctypes.c_int),
         "ckl_profile_collect": ([_P, ctypes.POINTER(KernelStat), ctypes.c_int,
                                  ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -349,6 +351,35 @@ class ChunkedKL:
             raise CKLError(code, "ckl_fwd_bwd_vocab_parallel") from group.error
         _check(code, "ckl_fwd_bwd_vocab_parallel")
         return (loss, dH, dW, lse, ell) if token_stats else (loss, dH, dW)
+
+    def forward_vocab_parallel(self, group: VocabGroup, H, W_shard, idx, logit, mask=None,
+                               chunk: int | None = None, token_stats: bool = False,
+                               sync: bool = True, stream=None):
+        """Loss only (identical on every rank); the handle's V is this rank's row count."""
+        T = self._inputs(H, W_shard, idx, logit, mask)
+        chunk = min(chunk or self.max_chunk, self.max_chunk)
+        n = _SZ()
+        _check(lib().ckl_vp_workspace_bytes(self._h, group.world, T, chunk, ctypes.byref(n)),
+               "ckl_vp_workspace_bytes")
+        ws = torch.empty(max(1, n.value), dtype=torch.uint8, device=self.device)
+        loss = torch.empty((), dtype=torch.float32, device=self.device)
+        lse = ell = None
+        if token_stats:
+            lse = torch.empty(T, dtype=torch.float32, device=self.device)
+            ell = torch.empty(T, dtype=torch.float32, device=self.device)
+        s = stream or torch.cuda.current_stream(self.device)
+        g, keep = group._c(self.device)
+        host = ctypes.c_float() if sync else None
+        group.error = None
+        code = lib().ckl_forward_vocab_parallel(
+            self._h, ctypes.byref(g), _ptr(H), _ptr(W_shard), _ptr(idx), _ptr(logit), _ptr(mask),
+            T, chunk, _ptr(loss), _ptr(lse), _ptr(ell), _ptr(ws), ws.numel(),
+            ctypes.c_void_p(s.cuda_stream), ctypes.byref(host) if sync else None)
+        del keep
+        if code == 9 and group.error is not None:
+            raise CKLError(code, "ckl_forward_vocab_parallel") from group.error
+        _check(code, "ckl_forward_vocab_parallel")
+        return (loss, lse, ell) if token_stats else loss
 
     def topk_cache(self, H, W, chunk: int | None = None, workspace=None, sync: bool = True,
                    stream=None):

@@ -228,7 +228,7 @@ ckl_status check_common(const ckl_ctx* h, const void* H, const void* W, const in
   return CKL_OK;
 }
 
-// `group` (vocabulary split over ranks, bf16 backward only) or nullptr.
+// `group` (vocabulary split over ranks, bf16 only) or nullptr.
 ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, const float* logit,
                const uint8_t* mask, int64_t T, int64_t chunk, float* loss, void* dH, float* dW,
                float* tok_lse, float* tok_loss, void* ws, size_t ws_bytes, cudaStream_t s,
@@ -293,7 +293,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
                                    reinterpret_cast<float*>(stats_all), (int64_t)Tc * 4, s);
         });
       }
-      if (!coll_rc) {
+      if (!coll_rc && backward) {
         coll_rc = L.collective(KID_VP_REDUCE, 0, [&] {
           return group->all_reduce_sum(group->user, dhf, (int64_t)Tc * d, s);
         });
@@ -625,18 +625,43 @@ ckl_status ckl_vp_workspace_bytes(ckl_handle h, int32_t world, int64_t T, int64_
   return CKL_OK;
 }
 
+namespace {
+ckl_status check_group(const ckl_ctx* h, const ckl_vocab_group* g, bool backward) {
+  if (!h || !g || g->world < 1 || g->rank < 0 || g->rank >= g->world || !g->all_gather ||
+      (backward && !g->all_reduce_sum) || g->v0 < 0 || g->V_total > INT32_MAX ||
+      g->v0 + h->V > g->V_total)
+    return CKL_ERR_INVALID_ARG;
+  if (h->dtype != CKL_BF16) return CKL_ERR_UNSUPPORTED;
+  return CKL_OK;
+}
+}  // namespace
+
+ckl_status ckl_forward_vocab_parallel(ckl_handle h, const ckl_vocab_group* g, const void* H,
+                                      const void* W_shard, const int32_t* topk_idx,
+                                      const float* topk_logit, const uint8_t* mask, int64_t T,
+                                      int64_t chunk, float* loss, float* token_lse,
+                                      float* token_loss, void* workspace, size_t workspace_bytes,
+                                      void* stream, float* loss_host) {
+  ckl_status st = check_group(h, g, false);
+  if (st != CKL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = run(h, H, W_shard, topk_idx, topk_logit, mask, T, chunk, loss, nullptr, nullptr, token_lse,
+           token_loss, workspace, workspace_bytes, s, false, g);
+  if (st != CKL_OK || !loss_host) return st;
+  DeviceGuard guard(h->device);
+  return sync_and_read(h, s, loss, loss_host);
+}
+
 ckl_status ckl_fwd_bwd_vocab_parallel(ckl_handle h, const ckl_vocab_group* g, const void* H,
                                       const void* W_shard, const int32_t* topk_idx,
                                       const float* topk_logit, const uint8_t* mask, int64_t T,
                                       int64_t chunk, float* loss, void* dH, float* dW_shard,
                                       float* token_lse, float* token_loss, void* workspace,
                                       size_t workspace_bytes, void* stream, float* loss_host) {
-  if (!h || !g || g->world < 1 || g->rank < 0 || g->rank >= g->world || !g->all_gather ||
-      !g->all_reduce_sum || g->v0 < 0 || g->V_total > INT32_MAX || g->v0 + h->V > g->V_total)
-    return CKL_ERR_INVALID_ARG;
-  if (h->dtype != CKL_BF16) return CKL_ERR_UNSUPPORTED;
+  ckl_status st = check_group(h, g, true);
+  if (st != CKL_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ckl_status st = run(h, H, W_shard, topk_idx, topk_logit, mask, T, chunk, loss, dH, dW_shard,
+  st = run(h, H, W_shard, topk_idx, topk_logit, mask, T, chunk, loss, dH, dW_shard,
                       token_lse, token_loss, workspace, workspace_bytes, s, true, g);
   if (st != CKL_OK || !loss_host) return st;
   DeviceGuard guard(h->device);

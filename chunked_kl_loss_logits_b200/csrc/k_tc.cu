@@ -520,9 +520,19 @@ cudaError_t launch_kind(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
   const int n_n = (p.N + L::BN - 1) / L::BN;
   const int n_tiles = n_m * n_n * (KIND == TcKind::DH ? p.n_split : 1);
   if (n_tiles <= 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       L::SMEM_BYTES);
+  // The shared-memory attribute is per device: set it once per device (bit per ordinal),
+  // so a call made during stream capture issues no attribute change.
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (!bit || !(attr_set.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set.fetch_or(bit, std::memory_order_release);
+  }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

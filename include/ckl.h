@@ -221,6 +221,17 @@ ckl_status ckl_fwd_bwd_vocab_parallel(ckl_handle h, const ckl_vocab_group* group
                                       float* token_lse, float* token_loss, void* workspace,
                                       size_t workspace_bytes, void* stream, float* loss_host);
 
+/* Loss only (no dH, dW), vocabulary split over ranks: one all-gather per chunk
+ * and no all-reduce (all_reduce_sum may be NULL). Loss, token_lse and
+ * token_loss as in ckl_fwd_bwd_vocab_parallel; the workspace of
+ * ckl_vp_workspace_bytes is enough. */
+ckl_status ckl_forward_vocab_parallel(ckl_handle h, const ckl_vocab_group* group, const void* H,
+                                      const void* W_shard, const int32_t* topk_idx,
+                                      const float* topk_logit, const uint8_t* mask, int64_t T,
+                                      int64_t chunk, float* loss, float* token_lse,
+                                      float* token_loss, void* workspace,
+                                      size_t workspace_bytes, void* stream, float* loss_host);
+
 /* Wait for `stream` and return the device-detected status of the calls enqueued
  * on it since the last synchronising call (clears it). */
 ckl_status ckl_sync_status(ckl_handle h, void* stream);

@@ -70,3 +70,5 @@ def test_null_handle_calls(L):
     assert L.ckl_vp_workspace_bytes(None, 2, 10, 4, ctypes.byref(n)) == 1
     assert L.ckl_fwd_bwd_vocab_parallel(None, None, *([None] * 5), 10, 4, *([None] * 6), 0, None,
                                         None) == 1
+    assert L.ckl_forward_vocab_parallel(None, None, *([None] * 5), 10, 4, *([None] * 4), 0, None,
+                                        None) == 1

@@ -60,7 +60,7 @@ class ThreadGroup:
         return ckl.VocabGroup(self.world, rank, V_total, v0, all_gather, all_reduce_sum)
 
 
-def run_group(x, world, chunk, shards=None):
+def run_group(x, world, chunk, shards=None, forward_only=False):
     T, d = x["H"].shape
     V = x["W"].shape[0]
     K = x["idx"].shape[1]
@@ -84,8 +84,9 @@ def run_group(x, world, chunk, shards=None):
             with torch.cuda.stream(s):
                 W_r = W[v0:v0 + n].contiguous()
                 s.synchronize()
-                res = h.fwd_bwd_vocab_parallel(tg.member(r, V, v0), H, W_r, idx, lg, mask,
-                                               chunk=chunk, token_stats=True)
+                fn = h.forward_vocab_parallel if forward_only else h.fwd_bwd_vocab_parallel
+                res = fn(tg.member(r, V, v0), H, W_r, idx, lg, mask, chunk=chunk,
+                         token_stats=True)
                 s.synchronize()
             out[r] = [t.cpu() for t in res]
             h.close()
@@ -257,3 +258,15 @@ def test_empty_input_makes_no_collective_call():
                                                                    device=dev),
                                             torch.zeros((0, 8), device=dev), chunk=32)
     assert calls == [] and float(loss) == 0.0 and torch.count_nonzero(dW) == 0
+
+
+def test_forward_only_group():
+    x = small_case(300, 128, 3000, 16, seed=37, dtype="bf16", teacher_var=3.0, ids="zipf",
+                   packing=True)
+    full, _, _ = run_group(x, 2, 128)
+    fwd, tg, _ = run_group(x, 2, 128, forward_only=True)
+    for r in range(2):
+        loss, lse, ell = fwd[r]
+        assert torch.equal(loss, full[r][0]) and torch.equal(lse, full[r][3])
+        assert torch.equal(ell, full[r][4])
+        assert [c[0] for c in tg.calls[r]] == ["gather"] * 3  # no all-reduce without a backward
