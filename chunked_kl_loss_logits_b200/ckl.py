@@ -440,11 +440,34 @@ class _ChunkedKLFn(torch.autograd.Function):
         return (dH * g.to(dH.dtype), (dW * g).to(ctx.w_dtype), None, None, None, None, None)
 
 
-def chunked_kl_loss(H, W, idx, logit, mask=None, chunk=None, handle: ChunkedKL | None = None):
-    """Autograd-friendly mean top-K forward KL; the gradients come from the fused call."""
+class _VocabParallelKLFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, H, W_shard, idx, logit, mask, handle, chunk, group):
+        loss, dH, dW = handle.fwd_bwd_vocab_parallel(group, H.detach(), W_shard.detach(), idx,
+                                                     logit, mask, chunk=chunk, sync=False)
+        ctx.save_for_backward(dH, dW)
+        ctx.w_dtype = W_shard.dtype
+        return loss
+
+    @staticmethod
+    def backward(ctx, g):
+        dH, dW = ctx.saved_tensors
+        return (dH * g.to(dH.dtype), (dW * g).to(ctx.w_dtype), None, None, None, None, None, None)
+
+
+def chunked_kl_loss(H, W, idx, logit, mask=None, chunk=None, handle: ChunkedKL | None = None,
+                    group: VocabGroup | None = None):
+    """Autograd-friendly mean top-K forward KL; the gradients come from the fused call.
+
+    With `group`, W is this rank's vocabulary rows (vocab_shards) and the loss is the
+    full-vocabulary one, identical on every rank; H's gradient is the full dH on
+    every rank and W's is this rank's rows.
+    """
     if handle is None:
         handle = ChunkedKL(W.shape[0], W.shape[1], idx.shape[1], dtype=W.dtype,
                            max_chunk=max(chunk or 4096, 1), device=W.device)
+    if group is not None:
+        return _VocabParallelKLFn.apply(H, W, idx, logit, mask, handle, chunk, group)
     return _ChunkedKLFn.apply(H, W, idx, logit, mask, handle, chunk)
 
 

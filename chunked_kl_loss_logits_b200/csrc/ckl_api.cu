@@ -268,7 +268,8 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
   float* dhf = group ? reinterpret_cast<float*>(base + P.off_dhf) : nullptr;
   const int V_all = group ? (int)group->V_total : (int)h->V;
   const int v0 = group ? (int)group->v0 : 0;
-  int coll_rc = 0;  // first failing collective's return code
+  int coll_rc = 0;          // first failing collective's return code
+  bool map_failed = false;  // a tensor map could not be encoded
 
   const int V = (int)h->V, d = (int)h->d, K = (int)h->K;
   const bool bf16 = h->dtype == CKL_BF16;
@@ -286,18 +287,31 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     const int Tc = (int)std::min<int64_t>(chunk, T - t0);
     const double zflops = 2.0 * Tc * (double)V * d;
     const unsigned char* Hc = static_cast<const unsigned char*>(H) + (size_t)t0 * d * esz;
-    if (err != cudaSuccess || coll_rc != 0) {
-      if (!coll_rc) {
-        coll_rc = L.collective(KID_VP_GATHER, 0, [&] {
-          return group->all_gather(group->user, reinterpret_cast<const float*>(stats),
-                                   reinterpret_cast<float*>(stats_all), (int64_t)Tc * 4, s);
-        });
-      }
-      if (!coll_rc && backward) {
-        coll_rc = L.collective(KID_VP_REDUCE, 0, [&] {
-          return group->all_reduce_sum(group->user, dhf, (int64_t)Tc * d, s);
-        });
-      }
+    // The chunk's collectives (group only): one all-gather, and with a backward
+    // one all-reduce. `drain` makes those not made yet, after a failure.
+    bool gathered = false, reduced = false;
+    auto gather = [&] {
+      gathered = true;
+      if (coll_rc) return;
+      coll_rc = L.collective(KID_VP_GATHER, (double)group->world * Tc * 16, [&] {
+        return group->all_gather(group->user, reinterpret_cast<const float*>(stats),
+                                 reinterpret_cast<float*>(stats_all), (int64_t)Tc * 4, s);
+      });
+    };
+    auto reduce = [&] {
+      reduced = true;
+      if (coll_rc || !backward) return;
+      coll_rc = L.collective(KID_VP_REDUCE, (double)Tc * d * 4, [&] {
+        return group->all_reduce_sum(group->user, dhf, (int64_t)Tc * d, s);
+      });
+    };
+    auto drain = [&] {
+      if (!group) return;
+      if (!gathered) gather();
+      if (!reduced) reduce();
+    };
+    if (err != cudaSuccess || coll_rc != 0 || map_failed) {
+      drain();
       continue;
     }
 
@@ -318,10 +332,13 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     TcMaps mz;
     if (bf16) {
       if (!make_map(h, &mz.a, Hc, d, Tc, (uint64_t)d * 2, 64, 128) ||
-          !make_map(h, &mz.b, W, d, V, (uint64_t)d * 2, 64, 128))
-        return CKL_ERR_CUDA;
-      if (backward && !make_map(h, &mz.c, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 32))
-        return CKL_ERR_CUDA;
+          !make_map(h, &mz.b, W, d, V, (uint64_t)d * 2, 64, 128) ||
+          (backward && !make_map(h, &mz.c, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 32))) {
+        map_failed = true;
+        if (!group) return CKL_ERR_CUDA;
+        drain();
+        continue;
+      }
       if (!backward) mz.c = mz.a;
     }
     chk(L(KID_LSE, zflops, store_e ? (double)Tc * V * 2 : 0, [&] {
@@ -342,12 +359,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     }));
     if (group) {
       // this rank's (max, sum, cross) per token to every rank; merged in rank order
-      if (!coll_rc) {
-        coll_rc = L.collective(KID_VP_GATHER, (double)group->world * Tc * 16, [&] {
-          return group->all_gather(group->user, reinterpret_cast<const float*>(stats),
-                                   reinterpret_cast<float*>(stats_all), (int64_t)Tc * 4, s);
-        });
-      }
+      gather();
       chk(L(KID_VP_MERGE, 0, (double)Tc * (group->world * 16.0 + 24.0), [&] {
         launch_vp_merge(t0, Tc, group->world, stats_all, mask, b, lse_all, ell_all, s);
       }));
@@ -384,8 +396,12 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
           !make_map(h, &mh.b, W, d, V, (uint64_t)d * 2, 64, 64) ||
           !make_map(h, &mw.a, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 64) ||
           !make_map(h, &mw.b, Hc, d, Tc, (uint64_t)d * 2, 64, 64) ||
-          !make_map(h, &mw.c, dW, d, V, (uint64_t)d * 4, 32, 32, true))
-        return CKL_ERR_CUDA;
+          !make_map(h, &mw.c, dW, d, V, (uint64_t)d * 4, 32, 32, true)) {
+        map_failed = true;
+        if (!group) return CKL_ERR_CUDA;
+        drain();
+        continue;
+      }
       mh.c = mh.a;
       chk(L(KID_DH, zflops, 0, [&] {
         TcLaunch p{};
@@ -403,11 +419,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
         chk(L(KID_DH_F32, 0, (double)Tc * d * (4.0 * P.n_split + 4.0), [&] {
           launch_dh_reduce_f32(b.dHp, P.n_split, (int64_t)Tc * d, dhf, s);
         }));
-        if (!coll_rc) {
-          coll_rc = L.collective(KID_VP_REDUCE, (double)Tc * d * 4, [&] {
-            return group->all_reduce_sum(group->user, dhf, (int64_t)Tc * d, s);
-          });
-        }
+        reduce();
         chk(L(KID_TO_BF16, 0, (double)Tc * d * 6.0, [&] {
           launch_f32_to_bf16(dhf, (int64_t)Tc * d, reinterpret_cast<uint16_t*>(dHc), s);
         }));
@@ -439,6 +451,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     std::fprintf(stderr, "ckl: CUDA error: %s\n", cudaGetErrorString(err));
     return CKL_ERR_CUDA;
   }
+  if (map_failed) return CKL_ERR_CUDA;
   if (coll_rc != 0) return CKL_ERR_COLLECTIVE;
   return CKL_OK;
 }

@@ -238,3 +238,37 @@ def test_launch_count_and_profiling():
     for k in ("lse_gemm", "scale_e", "dh_gemm", "dw_gemm", "teacher_topk"):
         assert stats[k]["launches"] == 2 and stats[k]["total_ms"] > 0
     assert stats["lse_gemm"]["flops"] == pytest.approx(2 * 256 * 1000 * 64)
+
+
+@pytest.mark.parametrize("T,d,V,K,chunk", [
+    (100, 8, 700, 8, 64),        # the smallest hidden size: one K-block, 56 zero-filled columns
+    (130, 24, 900, 12, 100),     # hidden size below one 64-wide K-block, not a power of two
+    (40, 64, 3000, 1024, 40),    # the largest K the teacher kernel takes
+])
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_extreme_sizes(T, d, V, K, chunk, dt):
+    x = small_case(T, d, V, K, seed=T + d + K, dtype=dt, teacher_var=3.0,
+                   ids="uniform" if K > V // 2 else "zipf")
+    run_and_compare(x, dt, chunk)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_one_word_vocabulary(dt):
+    # V = 1: every cached id is 0, so P = 1 there, softmax = 1, and the loss and
+    # both gradients are zero; in bf16 the gradient buffer holds bf16(1/N) before
+    # the 1/N of the teacher is subtracted, so G is zero only to within the bf16
+    # rounding of 1/N (relative 2^-9): |dH| <= 2^-8 max|W| / N, |dW| <= 2^-8 max|H|
+    x = small_case(70, 64, 1, 1, seed=61, dtype=dt)
+    x["idx"] = np.zeros((70, 4), dtype=np.int32)  # four slots, all holding the only id
+    x["logit"] = np.random.default_rng(61).standard_normal((70, 4)).astype(np.float32)
+    H, W, idx, logit, mask = upload(x, TORCH_DT[dt])
+    h = ckl.ChunkedKL(1, 64, 4, dtype=TORCH_DT[dt], max_chunk=32)
+    loss, dH, dW, lse, ell = h.fwd_bwd(H, W, idx, logit, mask, chunk=32, token_stats=True)
+    z = np.asarray(x["H"], np.float64) @ np.asarray(x["W"], np.float64).T
+    assert abs(loss.item()) <= 1e-6
+    rnd = 2.0 ** -8 if dt == "bf16" else 1e-6
+    N = x["H"].shape[0]
+    assert float(dH.float().abs().max()) <= rnd * np.abs(x["W"]).max() / N
+    assert float(dW.abs().max()) <= rnd * np.abs(x["H"]).max()
+    np.testing.assert_allclose(lse.cpu().numpy(), z[:, 0], rtol=1e-5, atol=1e-5)
+    h.close()

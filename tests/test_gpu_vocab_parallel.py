@@ -270,3 +270,22 @@ def test_forward_only_group():
         assert torch.equal(loss, full[r][0]) and torch.equal(lse, full[r][3])
         assert torch.equal(ell, full[r][4])
         assert [c[0] for c in tg.calls[r]] == ["gather"] * 3  # no all-reduce without a backward
+
+
+def test_autograd_with_a_group_of_one():
+    # the autograd wrapper routes through the vocabulary-parallel call
+    dev = torch.device("cuda", 0)
+    x = small_case(150, 64, 900, 8, seed=38, dtype="bf16")
+    H = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16).requires_grad_(True)
+    W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16).requires_grad_(True)
+    idx, lg = torch.from_numpy(x["idx"]).to(dev), torch.from_numpy(x["logit"]).to(dev)
+    calls = []
+    g = ckl.VocabGroup(1, 0, 900, 0, lambda s, r: (calls.append(1), r.copy_(s)),
+                       lambda b: calls.append(2))
+    loss = ckl.chunked_kl_loss(H, W, idx, lg, chunk=64, group=g)
+    (2.0 * loss).backward()
+    r = oracle.fwd_bwd(x["H"], x["W"], x["idx"], x["logit"])
+    assert abs(loss.item() - r["loss"]) <= 1e-3 * abs(r["loss"])
+    assert np.abs(H.grad.float().cpu().numpy() - 2 * r["dH"]).max() <= 2e-2 * np.abs(2 * r["dH"]).max()
+    assert np.abs(W.grad.float().cpu().numpy() - 2 * r["dW"]).max() <= 2e-2 * np.abs(2 * r["dW"]).max()
+    assert calls.count(1) == 3 and calls.count(2) == 3
