@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
                                         _I64, _P, _P, _P, _P, _P, _P, _SZ, _P, _P], ctypes.c_int),
         "ckl_forward_vocab_parallel": ([_P, ctypes.POINTER(_VocabGroupC), _P, _P, _P, _P, _P, _I64,
                                         _I64, _P, _P, _P, _P, _SZ, _P, _P], ctypes.c_int),
+        "ckl_selftest_wait_bound": ([_P, _P, ctypes.POINTER(_I64)], ctypes.c_int),
         "ckl_profile_enable": ([_P, ctypes.c_int, ctypes.c_int], ctypes.c_int),
         "ckl_profile_collect": ([_P, ctypes.POINTER(KernelStat), ctypes.c_int,
                                  ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -248,6 +249,14 @@ class ChunkedKL:
         return [{"name": arr[i].name.decode(), "launches": arr[i].launches,
                  "total_ms": arr[i].total_ms, "flops": arr[i].flops, "bytes": arr[i].bytes}
                 for i in range(min(n.value, 32))]
+
+    def selftest_wait_bound(self, stream=None):
+        """(status code, SM cycles waited) of the bounded-wait self-test; 6 (timeout) is a pass."""
+        s = stream or torch.cuda.current_stream(self.device)
+        cyc = _I64()
+        code = lib().ckl_selftest_wait_bound(self._h, ctypes.c_void_p(s.cuda_stream),
+                                             ctypes.byref(cyc))
+        return code, cyc.value
 
     def sync_status(self, stream=None):
         s = stream or torch.cuda.current_stream(self.device)

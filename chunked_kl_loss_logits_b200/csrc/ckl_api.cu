@@ -681,6 +681,24 @@ ckl_status ckl_fwd_bwd_vocab_parallel(ckl_handle h, const ckl_vocab_group* g, co
   return sync_and_read(h, s, loss, loss_host);
 }
 
+ckl_status ckl_selftest_wait_bound(ckl_handle h, void* stream, int64_t* cycles) {
+  if (!h) return CKL_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return CKL_ERR_CUDA;
+  cudaGetLastError();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // bytes 8..15 of the handle's 16-byte status block (device and pinned host)
+  long long* d_cyc = reinterpret_cast<long long*>(reinterpret_cast<unsigned char*>(h->d_status) + 8);
+  long long* h_cyc = reinterpret_cast<long long*>(reinterpret_cast<unsigned char*>(h->h_status) + 8);
+  launch_wait_selftest(h->d_status, d_cyc, s);
+  if (cudaGetLastError() != cudaSuccess) return CKL_ERR_CUDA;
+  if (cudaMemcpyAsync(h_cyc, d_cyc, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return CKL_ERR_CUDA;
+  const ckl_status st = sync_and_read(h, s, nullptr, nullptr);
+  if (cycles) *cycles = *h_cyc;
+  return st;
+}
+
 ckl_status ckl_sync_status(ckl_handle h, void* stream) {
   if (!h) return CKL_ERR_INVALID_ARG;
   DeviceGuard guard(h->device);

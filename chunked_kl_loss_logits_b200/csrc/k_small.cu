@@ -727,6 +727,27 @@ void launch_topk_select(const float2* cand, const int* cnt, int cap, int rows, i
                                                      status);
 }
 
+// Self-test of the bounded pipeline wait: one thread waits, with the same bounded
+// wait every pipeline kernel uses, on a freshly initialised mbarrier that nothing
+// arrives at (its phase 0 never completes). The wait must give up after its bound,
+// set ST_TIMEOUT and return; the kernel then exits. Completing is reported as
+// ST_INTERNAL (it cannot happen).
+__global__ void wait_bound_selftest_kernel(unsigned* status, long long* cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  abort_flag = 0;
+  const long long t0 = clock64();
+  const bool completed = mbar_wait(&bar, 0u, &abort_flag, status);
+  *cycles = clock64() - t0;
+  if (completed) atomicOr(status, (unsigned)ST_INTERNAL);
+}
+
+void launch_wait_selftest(unsigned* status, long long* cycles, cudaStream_t s) {
+  wait_bound_selftest_kernel<<<1, 32, 0, s>>>(status, cycles);
+}
+
 void launch_loss_finalize(const float* ell_all, const uint8_t* mask, int64_t T, Misc* misc,
                           float* loss, cudaStream_t s) {
   loss_finalize_kernel<<<1, kReduceThreads, 0, s>>>(ell_all, mask, T, misc, loss);

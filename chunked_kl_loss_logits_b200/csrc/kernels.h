@@ -62,6 +62,8 @@ void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int v0, 
 void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s);
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
                            cudaStream_t s);
+// One thread waits on a barrier nothing arrives at until the wait bound fires.
+void launch_wait_selftest(unsigned* status, long long* cycles, cudaStream_t s);
 // n_elem % 4 == 0
 void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out,
                           cudaStream_t s);

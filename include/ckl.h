@@ -232,6 +232,15 @@ ckl_status ckl_forward_vocab_parallel(ckl_handle h, const ckl_vocab_group* group
                                       float* token_loss, void* workspace,
                                       size_t workspace_bytes, void* stream, float* loss_host);
 
+/* Self-test of the device-side failure detection (the pages have no counterpart):
+ * one thread waits, with the bounded wait every pipeline kernel uses, on a barrier
+ * that nothing arrives at. The call waits for it and returns CKL_ERR_TIMEOUT when
+ * the bound fired as designed (4e9 SM cycles: about 2 s at the maximum clock,
+ * longer at lower clocks), with the cycles waited in *cycles (may be NULL); any
+ * other status means the mechanism failed. The status word is cleared and the
+ * handle stays usable. */
+ckl_status ckl_selftest_wait_bound(ckl_handle h, void* stream, int64_t* cycles);
+
 /* Wait for `stream` and return the device-detected status of the calls enqueued
  * on it since the last synchronising call (clears it). */
 ckl_status ckl_sync_status(ckl_handle h, void* stream);

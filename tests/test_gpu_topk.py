@@ -107,3 +107,21 @@ def test_cache_feeds_the_loss():
     q /= q.sum(1, keepdims=True)
     mass = np.take_along_axis(q, ids.cpu().numpy().astype(np.int64), 1).sum(1)
     np.testing.assert_allclose(ell.cpu().numpy(), -np.log(mass), rtol=1e-4, atol=1e-5)
+
+
+def test_k_equal_to_v_keeps_every_id_sorted():
+    x = small_case(50, 64, 200, 20, seed=11, dtype="bf16")
+    ids, lg = run(x, 200, 32)  # one vocabulary tile, K = V
+    z = np.asarray(x["H"], np.float64) @ np.asarray(x["W"], np.float64).T
+    for r in range(50):
+        assert sorted(ids[r].tolist()) == list(range(200))
+        assert np.all(np.diff(lg[r]) <= 0)
+        np.testing.assert_allclose(lg[r], z[r, ids[r]], rtol=0, atol=TOL)
+
+
+def test_cache_is_chunk_invariant():
+    x = small_case(300, 128, 5000, 24, seed=12, dtype="bf16")
+    a = run(x, 24, 300)
+    for chunk in (1, 77, 128):
+        b = run(x, 24, chunk)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
