@@ -149,7 +149,9 @@ WsPlan plan(const ckl_ctx* h, int64_t T, int64_t chunk, bool backward, int world
     p.off_zk = take((size_t)p.Tc * h->K * 4);
   }
   if (backward) {
-    p.off_G = take((size_t)p.Tc * p.ldG * (bf16 ? 2 : 4));
+    // bf16: blocked, 64 x 64 element blocks (8 KB); fp32: row-major, ldG
+    p.off_G = bf16 ? take((size_t)((p.Tc + 63) / 64) * ((h->V + 63) / 64) * 8192)
+                   : take((size_t)p.Tc * p.ldG * 4);
     if (bf16) p.off_dHp = take((size_t)p.n_split * p.Tc * h->d * 4);
   }
   if (world > 0) {
@@ -166,6 +168,24 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // 2-D tensor map (bf16, or fp32 when f32 is set): `inner` contiguous elements per
 // row, `outer` rows `row_bytes` apart, box of box_inner x box_outer, 128-byte
 // swizzle, zero fill outside the tensor (loads) / clipping (stores).
+// The bf16 gradient buffer of Tc tokens: 64 x 64 element blocks, 64 vocabulary ids
+// fastest inside a block, then 64 tokens; blocks vocabulary-block-major within a
+// token block. As a 4-D tensor (64, 64, vocabulary blocks, token blocks) with a
+// box of 64 ids x box_t tokens x 1 x box_tb token blocks.
+bool make_map_g(const ckl_ctx* h, CUtensorMap* m, const void* base, int64_t V, int64_t Tc,
+                uint32_t box_t, uint32_t box_tb) {
+  const cuuint64_t n_vb = (cuuint64_t)((V + 63) / 64), n_tb = (cuuint64_t)((Tc + 63) / 64);
+  const cuuint64_t dims[4] = {64, 64, n_vb, n_tb};
+  const cuuint64_t strides[3] = {128, 8192, n_vb * 8192};
+  const cuuint32_t box[4] = {64, box_t, 1, box_tb};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = h->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_map(const ckl_ctx* h, CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool f32 = false) {
   const cuuint64_t dims[2] = {inner, outer};
@@ -333,7 +353,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     if (bf16) {
       if (!make_map(h, &mz.a, Hc, d, Tc, (uint64_t)d * 2, 64, 128) ||
           !make_map(h, &mz.b, W, d, V, (uint64_t)d * 2, 64, 128) ||
-          (backward && !make_map(h, &mz.c, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 32))) {
+          (backward && !make_map_g(h, &mz.c, b.G, V, Tc, 32, 1))) {
         map_failed = true;
         if (!group) return CKL_ERR_CUDA;
         drain();
@@ -368,7 +388,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
 
     if (store_e) {
       chk(L(KID_SCALE, 0, (double)Tc * V * 4, [&] {
-        launch_scale_e(static_cast<uint16_t*>(b.G), P.ldG, Tc, V, b, s);
+        launch_scale_e(static_cast<uint16_t*>(b.G), Tc, V, b, s);
       }));
     } else {
       chk(L(KID_GRAD, zflops, (double)Tc * V * esz, [&] {
@@ -385,16 +405,16 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
       }));
     }
     chk(L(KID_FIXUP, 0, (double)Tc * K * (12.0 + 2 * esz), [&] {
-      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, v0, P.ldG, b, false, s);
+      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, v0, (V + 63) / 64, b, false, s);
       else launch_fixup<float>(idx, t0, Tc, K, V, v0, P.ldG, b, false, s);
     }));
 
     unsigned char* dHc = static_cast<unsigned char*>(dH) + (size_t)t0 * d * esz;
     if (bf16) {
       TcMaps mh, mw;
-      if (!make_map(h, &mh.a, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 128) ||
+      if (!make_map_g(h, &mh.a, b.G, V, Tc, 64, 2) ||
           !make_map(h, &mh.b, W, d, V, (uint64_t)d * 2, 64, 64) ||
-          !make_map(h, &mw.a, b.G, V, Tc, (uint64_t)P.ldG * 2, 64, 64) ||
+          !make_map_g(h, &mw.a, b.G, V, Tc, 64, 1) ||
           !make_map(h, &mw.b, Hc, d, Tc, (uint64_t)d * 2, 64, 64) ||
           !make_map(h, &mw.c, dW, d, V, (uint64_t)d * 4, 32, 32, true)) {
         map_failed = true;

@@ -340,40 +340,48 @@ __global__ void vp_merge_kernel(int64_t t0, int Tc, int world, const float4* __r
   finish_token(t0, i, M2, S, X, mask, tok, misc, cst, lse_all, ell_all);
 }
 
-// Stored-exp forward: the gradient buffer holds e = exp2(z log2e - m2_tile) in
-// bf16; turn it into G = gmul exp(z - lse) = e * gmul * exp2(m2_tile - lse log2e)
-// in place. Block (row i = blockIdx.x, 512 16-byte groups from blockIdx.y * 512):
-// each thread loads two 16-byte groups 256 apart before scaling either, so two
-// loads per thread are in flight.
-__global__ void __launch_bounds__(256) scale_e_kernel(uint16_t* __restrict__ G, int64_t ldG,
-                                                      int Tc, int V,
-                                                      const float2* __restrict__ part,
+// Stored-exp forward: the (blocked, bf16) gradient buffer holds
+// e = exp2(z log2e - m2_tile); turn it into G = gmul exp(z - lse)
+// = e * gmul * exp2(m2_tile - lse log2e) in place. One CUDA block per 64 x 64
+// element block of G (8 KB contiguous); each thread loads two 16-byte groups
+// (rows r and r + 32) before scaling either.
+__global__ void __launch_bounds__(256) scale_e_kernel(uint16_t* __restrict__ G, int n_vb, int Tc,
+                                                      int V, const float2* __restrict__ part,
                                                       const float4* __restrict__ cst) {
-  const int n8 = (V + 7) / 8;
-  const int i = blockIdx.x;
-  const int q0 = blockIdx.y * 512 + threadIdx.x, q1 = q0 + 256;
-  const float4 c = cst[i];
-  const float l2 = c.x * 1.4426950408889634f;
-  uint16_t* row = G + (int64_t)i * ldG;
+  const int vb = blockIdx.x, tb = blockIdx.y;
+  uint16_t* blk = G + ((int64_t)tb * n_vb + vb) * 4096;
+  const int c = (threadIdx.x & 7) * 8;            // first of the group's 8 columns
+  const int v = vb * 64 + c;
+  const int r0 = threadIdx.x >> 3;                // rows r0 and r0 + 32 of the block
+  const int t[2] = {tb * 64 + r0, tb * 64 + r0 + 32};
   uint4 x[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-  const int q[2] = {q0, q1};
+  if (v >= V) return;
 #pragma unroll
   for (int u = 0; u < 2; ++u)
-    if (q[u] < n8) x[u] = *reinterpret_cast<const uint4*>(row + (int64_t)q[u] * 8);
+    if (t[u] < Tc) x[u] = *reinterpret_cast<const uint4*>(blk + (r0 + 32 * u) * 64 + c);
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
-    if (q[u] >= n8) continue;
-    // 32 groups of 8 columns per 256-column vocabulary tile
-    const float f = c.y * ex2_approx(part[(int64_t)(q[u] >> 5) * Tc + i].x - l2);
+    if (t[u] >= Tc) continue;
+    const float4 cc = cst[t[u]];
+    const float f = cc.y * ex2_approx(part[(int64_t)(v >> 8) * Tc + t[u]].x -
+                                      cc.x * 1.4426950408889634f);
     uint4 y = x[u];
     y.x = pack_bf16x2(lo_bf16(y.x) * f, hi_bf16(y.x) * f);
     y.y = pack_bf16x2(lo_bf16(y.y) * f, hi_bf16(y.y) * f);
     y.z = pack_bf16x2(lo_bf16(y.z) * f, hi_bf16(y.z) * f);
     y.w = pack_bf16x2(lo_bf16(y.w) * f, hi_bf16(y.w) * f);
-    *reinterpret_cast<uint4*>(row + (int64_t)q[u] * 8) = y;
+    *reinterpret_cast<uint4*>(blk + (r0 + 32 * u) * 64 + c) = y;
   }
 }
 
+// Element (i, id) of the gradient buffer: fp32 row-major (ldG), bf16 blocked
+// (64 x 64 blocks, ld = the number of 64-wide vocabulary blocks).
+__device__ __forceinline__ int64_t g_off(const float*, int64_t i, int id, int64_t ld) {
+  return i * ld + id;
+}
+__device__ __forceinline__ int64_t g_off(const uint16_t*, int64_t i, int id, int64_t ld) {
+  return (((i >> 6) * ld + (id >> 6)) << 12) + ((i & 63) << 6) + (id & 63);
+}
 __device__ __forceinline__ void store_g(float* G, int64_t off, float v) { G[off] = v; }
 __device__ __forceinline__ void store_g(uint16_t* G, int64_t off, float v) {
   G[off] = f32_to_bf16(v);
@@ -400,7 +408,7 @@ __global__ void fixup_kernel(const int32_t* __restrict__ idx, int64_t t0, int Tc
   const int id = idx[t0 * K + e] - v0;
   if (id < 0 || id >= V) return;
   const float4 c = cst[i];
-  const int64_t off = i * ldG + id;
+  const int64_t off = g_off(G, i, id, ldG);
   const float g = overwrite ? c.y * expf(zk[e] - c.x) - c.z * P : load_g(G, off) - c.z * P;
   store_g(G, off, g);
 }
@@ -685,9 +693,10 @@ void launch_vp_merge(int64_t t0, int Tc, int world, const float4* stats_all, con
                                                       b.misc, b.cst, lse_all, ell_all);
 }
 
-void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s) {
-  const dim3 grid((unsigned)Tc, (unsigned)(((V + 7) / 8 + 511) / 512));
-  scale_e_kernel<<<grid, 256, 0, s>>>(G, ldG, Tc, V, b.part, b.cst);
+void launch_scale_e(uint16_t* G, int Tc, int V, const ChunkBufs& b, cudaStream_t s) {
+  const int n_vb = (V + 63) / 64;
+  const dim3 grid((unsigned)n_vb, (unsigned)((Tc + 63) / 64));
+  scale_e_kernel<<<grid, 256, 0, s>>>(G, n_vb, Tc, V, b.part, b.cst);
 }
 
 template <typename Tg>

@@ -71,6 +71,16 @@ template <> struct Cfg<TcKind::DW>   { static constexpr int BN = 256; static con
 template <> struct Cfg<TcKind::TKMAX>  { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
 template <> struct Cfg<TcKind::TKEMIT> { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
 
+// The bf16 gradient buffer is blocked: 64 x 64 element blocks (64 vocabulary ids
+// fastest, then 64 tokens; 8 KB contiguous), seen by TMA as the 4-D tensor
+// (64, 64, vocabulary blocks, token blocks). DH and DW read it as their A
+// operand (DH: K-major, 128 token rows = two blocks per box; DW: MN-major, one
+// block per 64-wide atom); LSE and GRAD write it from their epilogues.
+template <TcKind KIND>
+constexpr bool kAisG = KIND == TcKind::DH || KIND == TcKind::DW;
+template <TcKind KIND>
+constexpr bool kCisG = KIND == TcKind::LSE || KIND == TcKind::GRAD;
+
 template <TcKind KIND>
 struct Layout {
   static constexpr int BN = Cfg<KIND>::BN;
@@ -216,7 +226,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           unsigned char* sB = sA + L::A_BYTES;
           const uint32_t fbar = cluster_map(&full[stage], 0);
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::STAGE_BYTES);
-          if (!A_MN) {
+          if constexpr (kAisG<KIND> && !A_MN) {
+            // 128 token rows of one 64-wide vocabulary block: two token blocks
+            tma_load_4d_pair(sA, &tmA, fbar, 0, 0, kb, a_row0 >> 6);
+          } else if constexpr (kAisG<KIND>) {
+            // MN-major: one 64 (vocabulary) x 64 (token) block per atom
+#pragma unroll
+            for (int a = 0; a < BM / 64; ++a)
+              tma_load_4d_pair(sA + a * kAtomBytes, &tmA, fbar, 0, 0, (a_row0 >> 6) + a, kb);
+          } else if (!A_MN) {
             tma_load_2d_pair(sA, &tmA, fbar, kb * BK, a_row0);
           } else {
 #pragma unroll
@@ -295,8 +313,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char* stg = epi_smem + q * 2 * kStageBufBytes;  // this warp's two staging boxes
     int nstage = 0;                  // staging boxes this warp has filled so far
     // Fill staging box (nstage & 1) from this thread's row and hand it to TMA.
+    // Rows past the tensor are not stored, except in the gradient buffer: its last
+    // 64-token block is read whole by DW (rows past M against zero-filled H rows),
+    // so those rows must hold finite values, not what the workspace held before.
+    const int row_lim = kCisG<KIND> ? ((p.M + 63) & ~63) : p.M;
     auto stage_and_issue = [&](const uint4 (&chunks)[8], int c0, int c1, bool reduce) {
-      if (c1 >= p.M) return;  // every row of this warp's box lies past the tensor (warp-uniform)
+      if (c1 >= row_lim) return;  // every row of this warp's box is past the limit (warp-uniform)
       unsigned char* box = stg + (nstage & 1) * kStageBufBytes;
       if (lane == 0) bulk_wait_read<1>();  // the box's previous store has read it
       __syncwarp();
@@ -304,7 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        if (reduce) tma_reduce_add_2d(&tmC, box, c0, c1);
+        if constexpr (kCisG<KIND>) tma_store_4d(&tmC, box, 0, c1 & 63, c0 >> 6, c1 >> 6);
+        else if (reduce) tma_reduce_add_2d(&tmC, box, c0, c1);
         else tma_store_2d(&tmC, box, c0, c1);
         bulk_commit();
       }

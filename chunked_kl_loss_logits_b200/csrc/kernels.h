@@ -56,10 +56,12 @@ void launch_vp_merge(int64_t t0, int Tc, int world, const float4* stats_all, con
 // G at the cached ids. overwrite: G = gmul exp(z_k - lse) - s P_k (the gradient
 // contraction wrote gmul exp(z - lse) there); otherwise G -= s P_k in place.
 template <typename Tg>
+// ldG: fp32 row stride of G; bf16: the number of 64-wide vocabulary blocks (G blocked).
 void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int v0, int64_t ldG,
                   const ChunkBufs& b, bool overwrite, cudaStream_t s);
-// Stored-exp forward: G[i][v] = e[i][v] * gmul_i * exp2(m2[tile(v)][i] - lse_i log2 e), in place.
-void launch_scale_e(uint16_t* G, int64_t ldG, int Tc, int V, const ChunkBufs& b, cudaStream_t s);
+// Stored-exp forward: G[i][v] = e[i][v] * gmul_i * exp2(m2[tile(v)][i] - lse_i log2 e), in place
+// (G blocked, bf16).
+void launch_scale_e(uint16_t* G, int Tc, int V, const ChunkBufs& b, cudaStream_t s);
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
                            cudaStream_t s);
 // One thread waits on a barrier nothing arrives at until the wait bound fires.
