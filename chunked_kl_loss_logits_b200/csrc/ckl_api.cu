@@ -171,13 +171,13 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // The bf16 gradient buffer of Tc tokens: 64 x 64 element blocks, 64 vocabulary ids
 // fastest inside a block, then 64 tokens; blocks vocabulary-block-major within a
 // token block. As a 4-D tensor (64, 64, vocabulary blocks, token blocks) with a
-// box of 64 ids x box_t tokens x 1 x box_tb token blocks.
+// box of 64 ids x box_t tokens x box_vb vocabulary blocks x box_tb token blocks.
 bool make_map_g(const ckl_ctx* h, CUtensorMap* m, const void* base, int64_t V, int64_t Tc,
-                uint32_t box_t, uint32_t box_tb) {
+                uint32_t box_t, uint32_t box_vb, uint32_t box_tb) {
   const cuuint64_t n_vb = (cuuint64_t)((V + 63) / 64), n_tb = (cuuint64_t)((Tc + 63) / 64);
   const cuuint64_t dims[4] = {64, 64, n_vb, n_tb};
   const cuuint64_t strides[3] = {128, 8192, n_vb * 8192};
-  const cuuint32_t box[4] = {64, box_t, 1, box_tb};
+  const cuuint32_t box[4] = {64, box_t, box_vb, box_tb};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = h->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -353,7 +353,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     if (bf16) {
       if (!make_map(h, &mz.a, Hc, d, Tc, (uint64_t)d * 2, 64, 128) ||
           !make_map(h, &mz.b, W, d, V, (uint64_t)d * 2, 64, 128) ||
-          (backward && !make_map_g(h, &mz.c, b.G, V, Tc, 32, 1))) {
+          (backward && !make_map_g(h, &mz.c, b.G, V, Tc, 32, 1, 1))) {
         map_failed = true;
         if (!group) return CKL_ERR_CUDA;
         drain();
@@ -412,9 +412,9 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     unsigned char* dHc = static_cast<unsigned char*>(dH) + (size_t)t0 * d * esz;
     if (bf16) {
       TcMaps mh, mw;
-      if (!make_map_g(h, &mh.a, b.G, V, Tc, 64, 2) ||
+      if (!make_map_g(h, &mh.a, b.G, V, Tc, 64, 1, 2) ||
           !make_map(h, &mh.b, W, d, V, (uint64_t)d * 2, 64, 64) ||
-          !make_map_g(h, &mw.a, b.G, V, Tc, 64, 1) ||
+          !make_map_g(h, &mw.a, b.G, V, Tc, 64, 2, 1) ||
           !make_map(h, &mw.b, Hc, d, Tc, (uint64_t)d * 2, 64, 64) ||
           !make_map(h, &mw.c, dW, d, V, (uint64_t)d * 4, 32, 32, true)) {
         map_failed = true;

@@ -74,8 +74,9 @@ template <> struct Cfg<TcKind::TKEMIT> { static constexpr int BN = 256; static c
 // The bf16 gradient buffer is blocked: 64 x 64 element blocks (64 vocabulary ids
 // fastest, then 64 tokens; 8 KB contiguous), seen by TMA as the 4-D tensor
 // (64, 64, vocabulary blocks, token blocks). DH and DW read it as their A
-// operand (DH: K-major, 128 token rows = two blocks per box; DW: MN-major, one
-// block per 64-wide atom); LSE and GRAD write it from their epilogues.
+// operand (DH: K-major, 128 token rows = two token blocks per box; DW: MN-major,
+// two neighbouring vocabulary blocks per box, one per 64-wide atom); LSE and GRAD
+// write it from their epilogues.
 template <TcKind KIND>
 constexpr bool kAisG = KIND == TcKind::DH || KIND == TcKind::DW;
 template <TcKind KIND>
@@ -230,10 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 128 token rows of one 64-wide vocabulary block: two token blocks
             tma_load_4d_pair(sA, &tmA, fbar, 0, 0, kb, a_row0 >> 6);
           } else if constexpr (kAisG<KIND>) {
-            // MN-major: one 64 (vocabulary) x 64 (token) block per atom
-#pragma unroll
-            for (int a = 0; a < BM / 64; ++a)
-              tma_load_4d_pair(sA + a * kAtomBytes, &tmA, fbar, 0, 0, (a_row0 >> 6) + a, kb);
+            // MN-major: the CTA's two 64-wide atoms are two neighbouring (contiguous)
+            // blocks of one token block; one box, atom 1 landing kAtomBytes after atom 0
+            tma_load_4d_pair(sA, &tmA, fbar, 0, 0, a_row0 >> 6, kb);
           } else if (!A_MN) {
             tma_load_2d_pair(sA, &tmA, fbar, kb * BK, a_row0);
           } else {
