@@ -78,6 +78,10 @@ struct ckl_ctx {
   std::vector<cudaEvent_t> ev;  // pairs: ev[2i], ev[2i+1]
   int ev_used = 0;
   std::vector<ProfRec> recs;
+  // host-input calls: inputs are copied chunk by chunk on their own stream
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t copy_start = nullptr;
+  std::vector<cudaEvent_t> chunk_ready;
 };
 
 namespace {
@@ -248,11 +252,14 @@ ckl_status check_common(const ckl_ctx* h, const void* H, const void* W, const in
   return CKL_OK;
 }
 
-// `group` (vocabulary split over ranks, bf16 only) or nullptr.
+// `group` (vocabulary split over ranks, bf16 only) or nullptr. `ready` (or
+// nullptr): one event per chunk, recorded once that chunk's inputs (and, for
+// chunk 0, the mask) are on the device; the stream waits for it before using them.
 ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, const float* logit,
                const uint8_t* mask, int64_t T, int64_t chunk, float* loss, void* dH, float* dW,
                float* tok_lse, float* tok_loss, void* ws, size_t ws_bytes, cudaStream_t s,
-               bool backward, const ckl_vocab_group* group = nullptr) {
+               bool backward, const ckl_vocab_group* group = nullptr,
+               const cudaEvent_t* ready = nullptr) {
   ckl_status st = check_common(h, H, W, idx, logit, T, chunk, loss);
   if (st != CKL_OK) return st;
   if (backward) {
@@ -298,6 +305,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
   cudaError_t err = cudaSuccess;
   auto chk = [&](cudaError_t e) { if (e != cudaSuccess && err == cudaSuccess) err = e; };
 
+  if (ready && T > 0) chk(cudaStreamWaitEvent(s, ready[0], 0));
   chk(L(KID_MASK, 0, (double)T, [&] { launch_mask_count(mask, T, b.misc, s); }));
   if (backward && T == 0) chk(cudaMemsetAsync(dW, 0, (size_t)V * d * 4, s));
 
@@ -334,6 +342,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
       drain();
       continue;
     }
+    if (ready) chk(cudaStreamWaitEvent(s, ready[t0 / chunk], 0));
 
     if (bf16) {
       chk(L(KID_GATHER, 0, (double)Tc * K * 16.0, [&] {
@@ -586,6 +595,9 @@ ckl_status ckl_destroy(ckl_handle h) {
   if (!h) return CKL_OK;
   DeviceGuard guard(h->device);
   for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+  for (cudaEvent_t e : h->chunk_ready) cudaEventDestroy(e);
+  if (h->copy_start) cudaEventDestroy(h->copy_start);
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   if (h->d_status) cudaFree(h->d_status);
   if (h->h_status) cudaFreeHost(h->h_status);
   delete h;
@@ -628,27 +640,60 @@ ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t
                                  const void* W, int64_t T, int64_t chunk, float* loss, void* dH,
                                  float* dW, void* workspace, size_t workspace_bytes, void* stream,
                                  float* loss_host) {
-  if (!h || !loss_host || T < 0) return CKL_ERR_INVALID_ARG;
+  if (!h || !loss_host || T < 0 || chunk < 1) return CKL_ERR_INVALID_ARG;
   if (T > 0 && (!H_host || !idx_host || !logit_host || !H_dev || !idx_dev || !logit_dev))
     return CKL_ERR_INVALID_ARG;
   if (mask_host && !mask_dev) return CKL_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n_chunks = T > 0 ? (T + chunk - 1) / chunk : 0;
   {
     DeviceGuard guard(h->device);
     if (!guard.ok) return CKL_ERR_CUDA;
+    // The inputs go up chunk by chunk on the handle's copy stream, so chunk c + 1
+    // crosses the bus while chunk c computes. The copies start after everything
+    // already enqueued on `stream` (which may still read these device buffers).
+    if (!h->copy_stream &&
+        (cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking) != cudaSuccess ||
+         cudaEventCreateWithFlags(&h->copy_start, cudaEventDisableTiming) != cudaSuccess))
+      return CKL_ERR_CUDA;
+    while ((int64_t)h->chunk_ready.size() < n_chunks) {
+      cudaEvent_t e;
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return CKL_ERR_CUDA;
+      h->chunk_ready.push_back(e);
+    }
+    cudaStream_t c = h->copy_stream;
+    if (cudaEventRecord(h->copy_start, s) != cudaSuccess ||
+        cudaStreamWaitEvent(c, h->copy_start, 0) != cudaSuccess)
+      return CKL_ERR_CUDA;
     const size_t esz = h->dtype == CKL_BF16 ? 2 : 4;
-    if (T > 0) {
-      if (cudaMemcpyAsync(H_dev, H_host, (size_t)T * h->d * esz, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-          cudaMemcpyAsync(idx_dev, idx_host, (size_t)T * h->K * 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-          cudaMemcpyAsync(logit_dev, logit_host, (size_t)T * h->K * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return CKL_ERR_CUDA;
-      if (mask_host &&
-          cudaMemcpyAsync(mask_dev, mask_host, (size_t)T, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    if (T > 0 && mask_host &&
+        cudaMemcpyAsync(mask_dev, mask_host, (size_t)T, cudaMemcpyHostToDevice, c) != cudaSuccess)
+      return CKL_ERR_CUDA;
+    for (int64_t k = 0; k < n_chunks; ++k) {
+      const int64_t t0 = k * chunk, Tc = std::min<int64_t>(chunk, T - t0);
+      const size_t hb = (size_t)h->d * esz, kb = (size_t)h->K * 4;
+      if (cudaMemcpyAsync(static_cast<unsigned char*>(H_dev) + t0 * hb,
+                          static_cast<const unsigned char*>(H_host) + t0 * hb, Tc * hb,
+                          cudaMemcpyHostToDevice, c) != cudaSuccess ||
+          cudaMemcpyAsync(idx_dev + t0 * h->K, idx_host + t0 * h->K, Tc * kb,
+                          cudaMemcpyHostToDevice, c) != cudaSuccess ||
+          cudaMemcpyAsync(logit_dev + t0 * h->K, logit_host + t0 * h->K, Tc * kb,
+                          cudaMemcpyHostToDevice, c) != cudaSuccess ||
+          cudaEventRecord(h->chunk_ready[k], c) != cudaSuccess)
         return CKL_ERR_CUDA;
     }
   }
-  return ckl_fwd_bwd(h, H_dev, W, idx_dev, logit_dev, mask_host ? mask_dev : nullptr, T, chunk,
-                     loss, dH, dW, nullptr, nullptr, workspace, workspace_bytes, stream, loss_host);
+  ckl_status st = run(h, H_dev, W, idx_dev, logit_dev, mask_host ? mask_dev : nullptr, T, chunk,
+                      loss, dH, dW, nullptr, nullptr, workspace, workspace_bytes, s, true, nullptr,
+                      n_chunks ? h->chunk_ready.data() : nullptr);
+  if (st != CKL_OK) {
+    // the copies may still be running: do not return while they read the caller's buffers
+    DeviceGuard guard(h->device);
+    cudaStreamSynchronize(h->copy_stream);
+    return st;
+  }
+  DeviceGuard guard(h->device);
+  return sync_and_read(h, s, loss, loss_host);
 }
 
 ckl_status ckl_vp_workspace_bytes(ckl_handle h, int32_t world, int64_t T, int64_t chunk,

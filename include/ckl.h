@@ -112,10 +112,14 @@ ckl_status ckl_forward(ckl_handle h, const void* H, const void* W, const int32_t
 
 /* ckl_fwd_bwd with the per-step inputs in HOST memory: copies H_host, idx_host,
  * logit_host and mask_host (may be NULL) into the caller's device buffers H_dev,
- * idx_dev, logit_dev, mask_dev with one cudaMemcpyAsync each on `stream` (host
- * buffers should be pinned for the copies to be asynchronous), runs the fused
- * loss, copies the loss back to *loss_host and waits for the stream. W stays on
- * the device. Returns the device-detected status. */
+ * idx_dev, logit_dev, mask_dev, runs the fused loss, copies the loss back to
+ * *loss_host and waits. The copies run chunk by chunk (one cudaMemcpyAsync per
+ * tensor per chunk, the mask first) on a stream the handle creates on first use,
+ * after the work already enqueued on `stream`; chunk c's kernels wait for chunk
+ * c's copies only, so the next chunk crosses the bus while this one computes.
+ * Host buffers should be pinned for the copies to be asynchronous. W stays on the
+ * device. Returns the device-detected status; on an error no copy is still
+ * running when the call returns. */
 ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t* idx_host,
                                  const float* logit_host, const uint8_t* mask_host, void* H_dev,
                                  int32_t* idx_dev, float* logit_dev, uint8_t* mask_dev,

@@ -201,6 +201,32 @@ def test_from_host_matches_device_call():
     assert torch.equal(out[1], dH) and torch.equal(out[2], dW)
 
 
+def test_from_host_back_to_back_calls():
+    # the per-chunk copies of call n+1 must not overtake call n's kernels
+    xs = [small_case(333, 64, 1200, 12, seed=s, dtype="bf16", packing=(s == 81)) for s in (81, 82)]
+    dev = torch.device("cuda", 0)
+    h = ckl.ChunkedKL(1200, 64, 12, max_chunk=100)
+    W = torch.from_numpy(xs[0]["W"]).to(dev).to(torch.bfloat16)
+    refs, hosts = [], []
+    for x in xs:
+        H, _, idx, logit, mask = upload(x, torch.bfloat16)
+        refs.append(h.fwd_bwd(H, W, idx, logit, mask, chunk=100))
+        hosts.append(tuple(None if t is None else t.cpu().pin_memory() for t in (H, idx, logit, mask)))
+    stag = (torch.empty((333, 64), dtype=torch.bfloat16, device=dev),
+            torch.empty((333, 12), dtype=torch.int32, device=dev),
+            torch.empty((333, 12), dtype=torch.float32, device=dev),
+            torch.empty(333, dtype=torch.uint8, device=dev))
+    ws = h.workspace(333, 100)
+    s = torch.cuda.Stream(dev)
+    with torch.cuda.stream(s):
+        for k in (0, 1, 0, 1, 1, 0):
+            out = (torch.empty((), device=dev), torch.empty((333, 64), dtype=torch.bfloat16, device=dev),
+                   torch.empty((1200, 64), device=dev))
+            lv = h.fwd_bwd_from_host(*hosts[k], stag, W, 100, out, ws)
+            assert lv == refs[k][0].item()
+            assert torch.equal(out[1], refs[k][1]) and torch.equal(out[2], refs[k][2])
+
+
 def test_autograd_function():
     x = small_case(130, 64, 500, 8, seed=19, dtype="bf16")
     H, W, idx, logit, _ = upload(x, torch.bfloat16)
