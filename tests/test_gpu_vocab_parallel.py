@@ -289,3 +289,34 @@ def test_autograd_with_a_group_of_one():
     assert np.abs(H.grad.float().cpu().numpy() - 2 * r["dH"]).max() <= 2e-2 * np.abs(2 * r["dH"]).max()
     assert np.abs(W.grad.float().cpu().numpy() - 2 * r["dW"]).max() <= 2e-2 * np.abs(2 * r["dW"]).max()
     assert calls.count(1) == 3 and calls.count(2) == 3
+
+
+def test_nccl_group_of_one():
+    # the torch.distributed adapter on NCCL: collectives on device buffers wrapped
+    # from the library's pointers, ordered on the library's stream
+    import socket
+
+    import torch.distributed as dist
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dev = torch.device("cuda", 0)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=dev)
+    try:
+        x = small_case(300, 128, 3000, 16, seed=39, dtype="bf16", teacher_var=3.0, ids="zipf")
+        H = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
+        W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+        idx, lg = torch.from_numpy(x["idx"]).to(dev), torch.from_numpy(x["logit"]).to(dev)
+        g = ckl.torch_vocab_group(3000)
+        assert (g.world, g.rank, g.v0) == (1, 0, 0)
+        h = ckl.ChunkedKL(3000, 128, 16, max_chunk=128, device=dev)
+        s = torch.cuda.Stream(dev)
+        with torch.cuda.stream(s):
+            loss, dH, dW = h.fwd_bwd_vocab_parallel(g, H, W, idx, lg, chunk=128)
+        ref = h.fwd_bwd(H, W, idx, lg, chunk=128)
+        assert torch.equal(dH, ref[1]) and torch.equal(dW, ref[2])
+        torch.testing.assert_close(loss, ref[0], rtol=1e-6, atol=1e-7)
+        h.close()
+    finally:
+        dist.destroy_process_group()
