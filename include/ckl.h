@@ -18,22 +18,27 @@
  * dl_t/dz_v = M softmax(z)_v - P_v:
  *     dH = (mask/N) G W,    dW = sum_t (mask_t/N) G_t^T H_t.
  * The T x V logit tensor is never stored: the logits are produced tile by tile
- * on the tensor cores for the log-normaliser, and formed again chunk by chunk
- * (chunk tokens at a time) to build the analytic gradient: the README's fused
- * variant, which folds the output projection into the loss and never keeps the
- * logits of the whole sequence.
+ * on the tensor cores, chunk tokens at a time, and reduced to the log-normaliser
+ * in the tile's epilogue (the README's fused variant, which folds the output
+ * projection into the loss and never keeps the logits of the whole sequence).
+ * For the analytic gradient the default keeps exp(z - tile max) of the current
+ * chunk in the chunk-bounded gradient buffer; the README's design, which forms
+ * the chunk's logits again in the backward pass, is ckl_set_recompute(h, 1).
  *
  * Conventions for every entry point:
  *  - All matrices are dense, row-major, contiguous. H is T x d, W is V x d,
  *    topk_idx and topk_logit are T x K, mask is T bytes, dH is T x d, dW is V x d.
  *  - "device" pointers are CUDA device memory of the handle's device; the caller
- *    owns every buffer. The library allocates nothing during a call.
+ *    owns every buffer. The library allocates no device memory during a call
+ *    (ckl_fwd_bwd_from_host creates a stream and events on its first use).
  *  - H, W, dH have the handle's dtype (CKL_F32: float; CKL_BF16: bfloat16 bits).
  *    dW, topk_logit, loss and the per-token outputs are float32; topk_idx is int32.
  *  - H, W, dH, dW, topk_idx, topk_logit must be 16-byte aligned; the workspace
  *    256-byte aligned. mask has no alignment requirement.
  *  - stream is a cudaStream_t (NULL = legacy default stream); all work is
- *    enqueued on it in order. A handle must not be used by two calls at once.
+ *    enqueued on it in order (ckl_fwd_bwd_from_host adds its copies on a stream
+ *    of the handle, ordered after the work already on `stream`). A handle must
+ *    not be used by two calls at once.
  *  - Errors found on the host (bad sizes, null or misaligned pointers, a small
  *    workspace) return before anything is enqueued. Errors found on the device
  *    (a teacher id outside [0, V), a pipeline wait that exceeded its bound) set a
