@@ -56,3 +56,32 @@ def test_large_workload(name):
             assert ((dW - ref[2]).norm() / ref[2].norm()).item() <= 1e-5
         del loss, dH, dW, lse, ell
     h.close()
+
+
+def test_vocab_parallel_headline_shape():
+    # the 32K workload's head (V = 201088, d = 2880, K = 100), 4096 tokens in two
+    # chunks of 2048, the vocabulary split over two ranks run as threads: sampled
+    # rows against the oracle, identical results on both ranks, and the dW shards
+    # against the single-rank call
+    from tests.test_gpu_vocab_parallel import run_group
+    w = WORKLOADS["bf16_32k"]
+    x = make_inputs(w, T=4096)
+    rows = sample_rows(4096, 256, seed=w.seed)
+    r = oracle.sampled_rows(x["H"], x["W"], x["idx"], x["logit"], rows, x["mask"])
+    out, tg, shards = run_group(x, 2, 2048)
+    assert shards == ckl.vocab_shards(w.V, 2)
+    loss, dH, _, lse, ell = out[0]
+    for a, b in zip((loss, dH, lse, ell), (out[1][0], out[1][1], out[1][3], out[1][4])):
+        assert torch.equal(a, b)
+    rt = torch.from_numpy(rows)
+    assert rel_fro(f64(lse[rt]), r["lse"]) <= 1e-5
+    assert rel_fro(f64(ell[rt]), r["ell"]) <= TOL["bf16"]["loss"]
+    assert rel_fro(f64(dH[rt]), r["dH"]) <= TOL["bf16"]["grad"]
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=2048)
+    l1, dH1, dW1 = h.fwd_bwd(H, W, idx, logit, mask, chunk=2048)
+    assert rel(loss.item(), l1.item()) <= 1e-6
+    dW = torch.cat([o[2] for o in out])
+    assert ((dW - dW1.cpu()).norm() / dW1.cpu().norm()).item() <= 1e-3
+    assert ((dH.float() - dH1.cpu().float()).norm() / dH1.cpu().float().norm()).item() <= 1e-3
+    h.close()
