@@ -102,6 +102,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "power_w_max": max(power) if power else None,
+                "power_w_median": statistics.median(power) if power else None,
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
@@ -332,6 +333,9 @@ def run_ours(args, w, rank, world, local_rank):
                 "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": recorded_traffic(top["name"], w.name, chunk),
                 "peak_source": f"{peak_src} hbm_gbs", "avg_launch_ms": avg_ms}
+    if clocks.get("power_w_median"):
+        # board power under load x step time: the energy one step costs (the cap binds)
+        clocks["joules_per_step"] = clocks["power_w_median"] * step_ms / 1e3
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
