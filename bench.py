@@ -493,9 +493,10 @@ def run_compare(args, w):
         idx = torch.from_numpy(x["idx"]).to(dev)
         lg = torch.from_numpy(x["logit"]).to(dev)
         del x
-        # bytes held at the peak: bf16 z and its grad, several fp32 T x V tensors
-        est = {"dense_kl": T * w.V * (2 * 2 + 4 * 4), "forward_chunked": T * w.V * (2 * 2 + 4 * 2),
-               "ckl": 0}
+        # bytes per T x V element held at the peak, as measured at 4K-32K tokens
+        # (dense: bf16 z and its grad plus ~4 fp32 T x V tensors; forward-chunked: bf16 z,
+        # its grad and one fp32 chunk copy), with a margin
+        est = {"dense_kl": T * w.V * 23, "forward_chunked": T * w.V * 8.5, "ckl": 0}
         for method in ("dense_kl", "forward_chunked", "ckl"):
             rec = {"kind": "compare", "method": method, "workload": w.name, "T": T, "V": w.V,
                    "d": w.d, "K": w.K, "chunk": chunk if method != "dense_kl" else None}
