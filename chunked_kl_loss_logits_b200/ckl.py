@@ -87,6 +87,10 @@ def lib() -> ctypes.CDLL:
         "ckl_forward_vocab_parallel": ([_P, ctypes.POINTER(_VocabGroupC), _P, _P, _P, _P, _P, _I64,
                                         _I64, _P, _P, _P, _P, _SZ, _P, _P], ctypes.c_int),
         "ckl_selftest_wait_bound": ([_P, _P, ctypes.POINTER(_I64)], ctypes.c_int),
+        "ckl_topk_vp_workspace_bytes": ([_P, ctypes.c_int32, _I64, _I64, ctypes.POINTER(_SZ)],
+                                        ctypes.c_int),
+        "ckl_topk_cache_vocab_parallel": ([_P, ctypes.POINTER(_VocabGroupC), _P, _P, _I64, _I64,
+                                           _P, _P, _P, _SZ, _P, ctypes.c_int], ctypes.c_int),
         "ckl_profile_enable": ([_P, ctypes.c_int, ctypes.c_int], ctypes.c_int),
         "ckl_profile_collect": ([_P, ctypes.POINTER(KernelStat), ctypes.c_int,
                                  ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
@@ -412,6 +416,34 @@ class ChunkedKL:
         _check(lib().ckl_topk_cache(self._h, _ptr(H), _ptr(W), T, chunk, _ptr(idx), _ptr(logit),
                                     _ptr(workspace), workspace.numel(),
                                     ctypes.c_void_p(s.cuda_stream), int(sync)), "ckl_topk_cache")
+        return idx, logit
+
+    def topk_cache_vocab_parallel(self, group: VocabGroup, H, W_shard, chunk: int | None = None,
+                                  sync: bool = True, stream=None):
+        """Teacher top-K cache with the teacher's LM head split by vocabulary rows over
+        `group`: (ids int32 T x K, global; logits float32 T x K), the same on every
+        rank and the same as topk_cache with all of W on one rank."""
+        T = H.shape[0]
+        if H.dtype != self.dtype or W_shard.dtype != self.dtype or H.shape[1] != self.d or \
+                tuple(W_shard.shape) != (self.V, self.d):
+            raise ValueError("H must be T x d and W_shard V x d, in the handle's dtype")
+        chunk = min(chunk or self.max_chunk, self.max_chunk)
+        n = _SZ()
+        _check(lib().ckl_topk_vp_workspace_bytes(self._h, group.world, T, chunk, ctypes.byref(n)),
+               "ckl_topk_vp_workspace_bytes")
+        ws = torch.empty(max(1, n.value), dtype=torch.uint8, device=self.device)
+        idx = torch.empty((T, self.K), dtype=torch.int32, device=self.device)
+        logit = torch.empty((T, self.K), dtype=torch.float32, device=self.device)
+        s = stream or torch.cuda.current_stream(self.device)
+        g, keep = group._c(self.device)
+        group.error = None
+        code = lib().ckl_topk_cache_vocab_parallel(
+            self._h, ctypes.byref(g), _ptr(H), _ptr(W_shard), T, chunk, _ptr(idx), _ptr(logit),
+            _ptr(ws), ws.numel(), ctypes.c_void_p(s.cuda_stream), int(sync))
+        del keep
+        if code == 9 and group.error is not None:
+            raise CKLError(code, "ckl_topk_cache_vocab_parallel") from group.error
+        _check(code, "ckl_topk_cache_vocab_parallel")
         return idx, logit
 
     def fwd_bwd_from_host(self, H_host, idx_host, logit_host, mask_host, staging, W, chunk,

@@ -504,9 +504,12 @@ struct TopkPlan {
   int n_vt = 0;  // 256-wide vocabulary tiles
   int cap = 0;   // candidates per row: at most K tiles can beat the threshold
   size_t off_tbest = 0, off_theta = 0, off_cnt = 0, off_cand = 0, total = 0;
+  // vocabulary split over ranks: this rank's K best, packed, gathered, regrouped
+  size_t off_loc_idx = 0, off_loc_lg = 0, off_packed = 0, off_gathered = 0, off_cand2 = 0,
+         off_cnt2 = 0;
 };
 
-TopkPlan topk_plan(const ckl_ctx* h, int64_t T, int64_t chunk) {
+TopkPlan topk_plan(const ckl_ctx* h, int64_t T, int64_t chunk, int world = 0) {
   TopkPlan p;
   p.Tc = std::max<int64_t>(1, std::min(chunk, std::max<int64_t>(T, 1)));
   p.n_vt = (int)((h->V + 255) / 256);
@@ -517,6 +520,15 @@ TopkPlan topk_plan(const ckl_ctx* h, int64_t T, int64_t chunk) {
   p.off_theta = take((size_t)p.Tc * 8);
   p.off_cnt = take((size_t)p.Tc * 4);
   p.off_cand = take((size_t)p.Tc * p.cap * 8);
+  if (world > 0) {
+    const size_t tk = (size_t)p.Tc * h->K;
+    p.off_loc_idx = take(tk * 4);
+    p.off_loc_lg = take(tk * 4);
+    p.off_packed = take(tk * 8);
+    p.off_gathered = take(tk * 8 * world);
+    p.off_cand2 = take(tk * 8 * world);
+    p.off_cnt2 = take((size_t)p.Tc * 4);
+  }
   p.total = o;
   return p;
 }
@@ -792,9 +804,14 @@ ckl_status ckl_topk_workspace_bytes(ckl_handle h, int64_t T, int64_t chunk, size
   return CKL_OK;
 }
 
-ckl_status ckl_topk_cache(ckl_handle h, const void* H, const void* W, int64_t T, int64_t chunk,
-                          int32_t* topk_idx, float* topk_logit, void* workspace,
-                          size_t workspace_bytes, void* stream, int wait) {
+namespace {
+// The cache builder. With `group` (vocabulary split over ranks) each rank builds
+// the K best of its own rows into the extra buffers of the workspace, the pairs
+// are all-gathered per chunk, and every rank selects the final K of the world * K
+// candidates: the same result, bit for bit, as one rank holding all of W.
+ckl_status topk_run(ckl_ctx* h, const ckl_vocab_group* group, const void* H, const void* W,
+                    int64_t T, int64_t chunk, int32_t* topk_idx, float* topk_logit,
+                    void* workspace, size_t workspace_bytes, void* stream, int wait) {
   if (!h || !W || T < 0 || chunk < 1 || chunk > h->max_chunk || chunk > INT32_MAX)
     return CKL_ERR_INVALID_ARG;
   if (T > 0 && (!H || !topk_idx || !topk_logit)) return CKL_ERR_INVALID_ARG;
@@ -802,7 +819,7 @@ ckl_status ckl_topk_cache(ckl_handle h, const void* H, const void* W, int64_t T,
   if (!aligned(W, 16) || (H && !aligned(H, 16)) || (topk_idx && !aligned(topk_idx, 4)) ||
       (topk_logit && !aligned(topk_logit, 4)))
     return CKL_ERR_ALIGNMENT;
-  const TopkPlan P = topk_plan(h, T, chunk);
+  const TopkPlan P = topk_plan(h, T, chunk, group ? group->world : 0);
   if (T > 0 && (!workspace || !aligned(workspace, 256) || workspace_bytes < P.total))
     return CKL_ERR_WORKSPACE;
   DeviceGuard guard(h->device);
@@ -815,17 +832,42 @@ ckl_status ckl_topk_cache(ckl_handle h, const void* H, const void* W, int64_t T,
   float2* theta = reinterpret_cast<float2*>(base + P.off_theta);
   int* cnt = reinterpret_cast<int*>(base + P.off_cnt);
   float2* cand = reinterpret_cast<float2*>(base + P.off_cand);
+  int32_t* loc_idx = group ? reinterpret_cast<int32_t*>(base + P.off_loc_idx) : nullptr;
+  float* loc_lg = group ? reinterpret_cast<float*>(base + P.off_loc_lg) : nullptr;
+  float2* packed = group ? reinterpret_cast<float2*>(base + P.off_packed) : nullptr;
+  float2* gathered = group ? reinterpret_cast<float2*>(base + P.off_gathered) : nullptr;
+  float2* cand2 = group ? reinterpret_cast<float2*>(base + P.off_cand2) : nullptr;
+  int* cnt2 = group ? reinterpret_cast<int*>(base + P.off_cnt2) : nullptr;
   Launcher L{h, s};
   cudaError_t err = cudaSuccess;
+  int coll_rc = 0;
+  bool map_failed = false;
   auto chk = [&](cudaError_t e) { if (e != cudaSuccess && err == cudaSuccess) err = e; };
-  for (int64_t t0 = 0; t0 < T && err == cudaSuccess; t0 += chunk) {
+  // With a group every chunk makes its one all-gather, also after a kernel
+  // failure (the ranks' calls stay matched); only the kernels are skipped.
+  for (int64_t t0 = 0; t0 < T && (err == cudaSuccess || group); t0 += chunk) {
     const int Tc = (int)std::min<int64_t>(chunk, T - t0);
     const double zflops = 2.0 * Tc * (double)V * d;
     const unsigned char* Hc = static_cast<const unsigned char*>(H) + (size_t)t0 * d * 2;
+    auto gather = [&] {
+      if (coll_rc) return;
+      coll_rc = L.collective(KID_VP_GATHER, (double)group->world * Tc * K * 8, [&] {
+        return group->all_gather(group->user, reinterpret_cast<const float*>(packed),
+                                 reinterpret_cast<float*>(gathered), (int64_t)Tc * K * 2, s);
+      });
+    };
+    if (err != cudaSuccess || coll_rc != 0 || map_failed) {
+      gather();
+      continue;
+    }
     TcMaps m;
     if (!make_map(h, &m.a, Hc, d, Tc, (uint64_t)d * 2, 64, 128) ||
-        !make_map(h, &m.b, W, d, V, (uint64_t)d * 2, 64, 128))
-      return CKL_ERR_CUDA;
+        !make_map(h, &m.b, W, d, V, (uint64_t)d * 2, 64, 128)) {
+      map_failed = true;
+      if (!group) return CKL_ERR_CUDA;
+      gather();
+      continue;
+    }
     m.c = m.a;
     chk(cudaMemsetAsync(cnt, 0, (size_t)Tc * 4, s));
     chk(L(KID_TKMAX, zflops, 0, [&] {
@@ -845,16 +887,57 @@ ckl_status ckl_topk_cache(ckl_handle h, const void* H, const void* W, int64_t T,
       launch_tc(m, p, s);
     }));
     chk(L(KID_TKSELECT, 0, (double)Tc * K * 8, [&] {
-      launch_topk_select(cand, cnt, P.cap, Tc, K, topk_idx + t0 * K, topk_logit + t0 * K,
-                         h->d_status, s);
+      launch_topk_select(cand, cnt, P.cap, Tc, K, group ? loc_idx : topk_idx + t0 * K,
+                         group ? loc_lg : topk_logit + t0 * K, h->d_status, s);
     }));
+    if (group) {
+      chk(L(KID_TKSELECT, 0, (double)Tc * K * 16, [&] {
+        launch_topk_pack(loc_idx, loc_lg, (int64_t)Tc * K, (int)group->v0, packed, s);
+      }));
+      gather();
+      chk(L(KID_TKSELECT, 0, (double)group->world * Tc * K * 16, [&] {
+        launch_topk_regroup(gathered, group->world, Tc, K, cand2, cnt2, s);
+      }));
+      chk(L(KID_TKSELECT, 0, (double)group->world * Tc * K * 8, [&] {
+        launch_topk_select(cand2, cnt2, group->world * K, Tc, K, topk_idx + t0 * K,
+                           topk_logit + t0 * K, h->d_status, s);
+      }));
+    }
   }
   if (err != cudaSuccess) {
     std::fprintf(stderr, "ckl: CUDA error: %s\n", cudaGetErrorString(err));
     return CKL_ERR_CUDA;
   }
+  if (map_failed) return CKL_ERR_CUDA;
+  if (coll_rc != 0) return CKL_ERR_COLLECTIVE;
   if (!wait) return CKL_OK;
   return sync_and_read(h, s, nullptr, nullptr);
+}
+}  // namespace
+
+ckl_status ckl_topk_cache(ckl_handle h, const void* H, const void* W, int64_t T, int64_t chunk,
+                          int32_t* topk_idx, float* topk_logit, void* workspace,
+                          size_t workspace_bytes, void* stream, int wait) {
+  return topk_run(h, nullptr, H, W, T, chunk, topk_idx, topk_logit, workspace, workspace_bytes,
+                  stream, wait);
+}
+
+ckl_status ckl_topk_vp_workspace_bytes(ckl_handle h, int32_t world, int64_t T, int64_t chunk,
+                                       size_t* bytes) {
+  if (!h || !bytes || world < 1 || T < 0 || chunk < 1) return CKL_ERR_INVALID_ARG;
+  *bytes = topk_plan(h, T, chunk, world).total;
+  return CKL_OK;
+}
+
+ckl_status ckl_topk_cache_vocab_parallel(ckl_handle h, const ckl_vocab_group* g, const void* H,
+                                         const void* W_shard, int64_t T, int64_t chunk,
+                                         int32_t* topk_idx, float* topk_logit, void* workspace,
+                                         size_t workspace_bytes, void* stream, int wait) {
+  if (!h || !g || g->world < 1 || g->rank < 0 || g->rank >= g->world || !g->all_gather ||
+      g->v0 < 0 || g->V_total > INT32_MAX || g->v0 + h->V > g->V_total)
+    return CKL_ERR_INVALID_ARG;
+  return topk_run(h, g, H, W_shard, T, chunk, topk_idx, topk_logit, workspace, workspace_bytes,
+                  stream, wait);
 }
 
 ckl_status ckl_set_recompute(ckl_handle h, int recompute) {

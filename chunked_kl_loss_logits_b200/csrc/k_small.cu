@@ -724,6 +724,39 @@ void launch_f32_to_bf16(const float* in, int64_t n_elem, uint16_t* out, cudaStre
   f32_to_bf16_kernel<<<blocks_for(n_elem / 4, 256), 256, 0, s>>>(in, n_elem, out);
 }
 
+// Vocabulary split over ranks (top-K cache): this rank's K best of each row as
+// (logit, global id) pairs, ids shifted by the rank's first row v0.
+__global__ void topk_pack_kernel(const int32_t* __restrict__ idx, const float* __restrict__ lg,
+                                 int64_t n, int v0, float2* __restrict__ out) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < n) out[e] = make_float2(lg[e], __int_as_float(idx[e] + v0));
+}
+
+// The gathered pairs are rank-major (world x rows x K); the select wants each
+// row's world * K candidates together, with their count.
+__global__ void topk_regroup_kernel(const float2* __restrict__ gathered, int world, int rows, int K,
+                                    float2* __restrict__ cand, int* __restrict__ cnt) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t per_rank = (int64_t)rows * K;
+  if (e >= per_rank * world) return;
+  const int r = (int)(e / per_rank);
+  const int64_t q = e - r * per_rank;
+  const int row = (int)(q / K), k = (int)(q - (int64_t)row * K);
+  cand[(int64_t)row * world * K + (int64_t)r * K + k] = gathered[e];
+  if (r == 0 && k == 0) cnt[row] = world * K;
+}
+
+void launch_topk_pack(const int32_t* idx, const float* lg, int64_t n, int v0, float2* out,
+                      cudaStream_t s) {
+  topk_pack_kernel<<<blocks_for(n, 256), 256, 0, s>>>(idx, lg, n, v0, out);
+}
+
+void launch_topk_regroup(const float2* gathered, int world, int rows, int K, float2* cand, int* cnt,
+                         cudaStream_t s) {
+  topk_regroup_kernel<<<blocks_for((int64_t)world * rows * K, 256), 256, 0, s>>>(
+      gathered, world, rows, K, cand, cnt);
+}
+
 void launch_topk_threshold(const float2* tbest, int n_vt, int rows, int K, float2* theta,
                            cudaStream_t s) {
   topk_threshold_kernel<<<blocks_for(rows, kThreshWarps), kThreshWarps * 32, 0, s>>>(

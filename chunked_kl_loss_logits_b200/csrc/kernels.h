@@ -66,6 +66,12 @@ void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16
                            cudaStream_t s);
 // One thread waits on a barrier nothing arrives at until the wait bound fires.
 void launch_wait_selftest(unsigned* status, long long* cycles, cudaStream_t s);
+// Top-K cache with the vocabulary split over ranks: pack this rank's K best as
+// (logit, global id); regroup the gathered pairs per row for the final select.
+void launch_topk_pack(const int32_t* idx, const float* lg, int64_t n, int v0, float2* out,
+                      cudaStream_t s);
+void launch_topk_regroup(const float2* gathered, int world, int rows, int K, float2* cand, int* cnt,
+                         cudaStream_t s);
 // n_elem % 4 == 0
 void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out,
                           cudaStream_t s);

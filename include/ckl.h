@@ -250,6 +250,22 @@ ckl_status ckl_forward_vocab_parallel(ckl_handle h, const ckl_vocab_group* group
  * handle stays usable. */
 ckl_status ckl_selftest_wait_bound(ckl_handle h, void* stream, int64_t* cycles);
 
+/* The top-K cache builder for a teacher whose LM head is split by vocabulary rows
+ * over a group (ckl_vocab_group as above; this handle's V = the rank's rows, and
+ * K <= V). Each rank builds the K best of its own rows per chunk; the group
+ * all-gathers the (logit, global id) pairs (one all-gather per chunk, world x
+ * chunk x K x 8 bytes; all_reduce_sum is not used and may be NULL) and every rank
+ * selects the final K of the world * K candidates, so every rank gets the cache
+ * ckl_topk_cache would give one rank holding all of W, bit for bit. Workspace:
+ * ckl_topk_vp_workspace_bytes. Errors and matched collectives as in
+ * ckl_fwd_bwd_vocab_parallel. */
+ckl_status ckl_topk_vp_workspace_bytes(ckl_handle h, int32_t world, int64_t T, int64_t chunk,
+                                       size_t* bytes);
+ckl_status ckl_topk_cache_vocab_parallel(ckl_handle h, const ckl_vocab_group* group, const void* H,
+                                         const void* W_shard, int64_t T, int64_t chunk,
+                                         int32_t* topk_idx, float* topk_logit, void* workspace,
+                                         size_t workspace_bytes, void* stream, int wait);
+
 /* Wait for `stream` and return the device-detected status of the calls enqueued
  * on it since the last synchronising call (clears it). */
 ckl_status ckl_sync_status(ckl_handle h, void* stream);

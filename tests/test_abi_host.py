@@ -68,6 +68,9 @@ def test_null_handle_calls(L):
     assert L.ckl_destroy(None) == 0
     assert L.ckl_profile_enable(None, 1, 16) == 1
     assert L.ckl_selftest_wait_bound(None, None, None) == 1
+    assert L.ckl_topk_vp_workspace_bytes(None, 2, 10, 4, ctypes.byref(n)) == 1
+    assert L.ckl_topk_cache_vocab_parallel(None, None, None, None, 10, 4, None, None, None, 0,
+                                           None, 0) == 1
     assert L.ckl_vp_workspace_bytes(None, 2, 10, 4, ctypes.byref(n)) == 1
     assert L.ckl_fwd_bwd_vocab_parallel(None, None, *([None] * 5), 10, 4, *([None] * 6), 0, None,
                                         None) == 1

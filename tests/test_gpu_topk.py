@@ -125,3 +125,68 @@ def test_cache_is_chunk_invariant():
     for chunk in (1, 77, 128):
         b = run(x, 24, chunk)
         assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def run_cache_group(x, K, chunk, world):
+    """The cache built by `world` ranks (threads) holding vocab_shards of W."""
+    import threading
+
+    from tests.test_gpu_vocab_parallel import ThreadGroup
+    T, d = x["H"].shape
+    V = x["W"].shape[0]
+    dev = torch.device("cuda", 0)
+    H = torch.from_numpy(x["H"]).to(dev).to(torch.bfloat16)
+    W = torch.from_numpy(x["W"]).to(dev).to(torch.bfloat16)
+    torch.cuda.synchronize(dev)
+    shards = ckl.vocab_shards(V, world)
+    tg = ThreadGroup(world)
+    out, errs = [None] * world, []
+
+    def rank_main(r):
+        try:
+            torch.cuda.set_device(dev)
+            v0, n = shards[r]
+            h = ckl.ChunkedKL(n, d, K, max_chunk=chunk, device=dev)
+            s = torch.cuda.Stream(dev)
+            with torch.cuda.stream(s):
+                W_r = W[v0:v0 + n].contiguous()
+                s.synchronize()
+                ids, lg = h.topk_cache_vocab_parallel(tg.member(r, V, v0), H, W_r, chunk=chunk)
+                s.synchronize()
+            out[r] = (ids.cpu(), lg.cpu())
+            h.close()
+        except Exception as e:
+            errs.append(e)
+            tg.barrier.abort()
+
+    th = [threading.Thread(target=rank_main, args=(r,)) for r in range(world)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join(300)
+    assert not errs, errs
+    return out, tg
+
+
+@pytest.mark.parametrize("world,T,d,V,K,chunk", [
+    (2, 300, 128, 5000, 24, 128),
+    (3, 257, 64, 5000, 24, 100),    # uneven shards (1792, 1792, 1416 rows)
+])
+def test_vocab_parallel_cache_equals_single_rank(world, T, d, V, K, chunk):
+    x = small_case(T, d, V, K, seed=world + T, dtype="bf16")
+    out, tg = run_cache_group(x, K, chunk, world)
+    ref_ids, ref_lg = run(x, K, chunk)
+    for ids, lg in out:
+        assert np.array_equal(ids.numpy(), ref_ids) and np.array_equal(lg.numpy(), ref_lg)
+    n_chunks = (T + chunk - 1) // chunk
+    for calls in tg.calls:
+        assert [c[0] for c in calls] == ["gather"] * n_chunks
+
+
+def test_vocab_parallel_cache_headline_shape():
+    w = WORKLOADS["bf16_32k"]
+    x = make_inputs(w, T=512)
+    out, _ = run_cache_group(x, w.K, 256, 2)
+    ref_ids, ref_lg = run(x, w.K, 256)
+    for ids, lg in out:
+        assert np.array_equal(ids.numpy(), ref_ids) and np.array_equal(lg.numpy(), ref_lg)
