@@ -109,7 +109,7 @@ class ClockSampler:
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_bf16_32k.md")
 # The sources of the tensor-core kernels whose DRAM traffic the summary records.
 KERNEL_SOURCES = ("chunked_kl_loss_logits_b200/csrc/k_tc.cu", "chunked_kl_loss_logits_b200/csrc/common.cuh",
-                  "chunked_kl_loss_logits_b200/csrc/kernels.h")
+                  "chunked_kl_loss_logits_b200/csrc/k_tc.h")
 
 
 def kernel_source_hash() -> str:

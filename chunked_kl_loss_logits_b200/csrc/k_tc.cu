@@ -45,7 +45,7 @@
 #include <atomic>
 
 #include "common.cuh"
-#include "kernels.h"
+#include "k_tc.h"
 
 namespace ckl {
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "k_tc.h"
+
 namespace ckl {
 
 // Per-token values of the chunk being processed, in the workspace.
@@ -97,40 +99,5 @@ void launch_simt_gemm(const float* A, int64_t sam, int64_t sak, const float* B, 
                       cudaStream_t s);
 constexpr int kSimtTile = 64;
 
-// ---- bf16 tcgen05 path (k_tc.cu)
-struct TcMaps {
-  CUtensorMap a, b, c;  // operands A and B; c = epilogue store target (G or dW)
-};
-enum class TcKind : int { LSE = 0, GRAD = 1, DH = 2, DW = 3, TKMAX = 4, TKEMIT = 5 };
-struct TcLaunch {
-  TcKind kind;
-  int M, N, n_kb;  // output rows, output cols, 64-wide blocks along the contraction
-  int n_split;     // DH only: contraction splits (>= 1)
-  int V;           // LSE / GRAD: number of valid vocabulary columns
-  float2* part;    // LSE
-  int part_ld;     // LSE: rows of one vocabulary tile's partials (= Tc)
-  const int32_t* sid;  // LSE: sorted cached ids per row (Tc x K)
-  const float* sp;     // LSE: their teacher probabilities
-  float* xpart;        // LSE: per-tile partial cross term, same layout as part
-  int K;
-  int store_e;     // LSE: also store exp(z - tile max) in bf16 through map c
-  const float4* cst;  // GRAD
-  uint16_t* G;        // GRAD
-  int64_t ldG;        // GRAD
-  float* dHp;         // DH
-  float* dW;          // DW
-  int first;          // DW: overwrite instead of accumulate
-  // teacher top-K cache: TKMAX writes each row's best (logit, id) per vocabulary
-  // tile into `part` (id stored as float bits); TKEMIT appends every (logit, id)
-  // at least as good as the row's threshold `theta` to the row's candidate list.
-  const float2* theta;
-  float2* cand;
-  int* cand_cnt;
-  int cand_cap;
-  unsigned* status;
-  int num_sms;
-};
-int tc_bn(TcKind k);  // output tile width of a kind
-cudaError_t launch_tc(const TcMaps& maps, const TcLaunch& p, cudaStream_t s);
-
+// ---- bf16 tcgen05 path (k_tc.cu): declared in k_tc.h
 }  // namespace ckl
