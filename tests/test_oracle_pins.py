@@ -309,19 +309,38 @@ def _mut_student_transposed(H_rows, W):
     return z[:, ::-1].copy()
 
 
+def _mut_unpooled(idx, p):
+    return np.asarray(p, dtype=np.float64).copy()  # a repeated id keeps only its own slot
+
+
+def _mut_mask_ignored(mask, T):
+    return _orig_token_scale(None, T)
+
+
 _orig_token_loss = O.token_loss
 _orig_grad_logits = O.grad_logits
 _orig_student_logits = O.student_logits
+_orig_token_scale = O.token_scale
 
 
-@pytest.mark.parametrize("name,fn", [("token_loss", _mut_drop_lse), ("token_loss", _mut_cross_sign),
-                                     ("grad_logits", _mut_grad_no_p),
-                                     ("grad_logits", _mut_grad_shift_idx),
-                                     ("student_logits", _mut_student_transposed)])
+PLANTED = [("token_loss", _mut_drop_lse), ("token_loss", _mut_cross_sign),
+           ("grad_logits", _mut_grad_no_p), ("grad_logits", _mut_grad_shift_idx),
+           ("student_logits", _mut_student_transposed), ("merged_probs", _mut_unpooled),
+           ("token_scale", _mut_mask_ignored)]
+
+
+@pytest.mark.parametrize("name,fn", PLANTED)
+def test_brute_force_pin_catches_every_planted_mistake(monkeypatch, name, fn):
+    monkeypatch.setattr(O, name, fn)
+    with pytest.raises(AssertionError):
+        test_brute_force_loops()
+
+
+@pytest.mark.parametrize("name,fn", PLANTED[:5])
 def test_pins_catch_planted_mistakes(monkeypatch, name, fn):
     monkeypatch.setattr(O, name, fn)
     pins = [lambda: test_dense_reconstruction(1, True), lambda: test_torch_kl_div_autograd(3, False),
-            test_finite_differences, test_gradient_rows_sum_to_zero]
+            test_finite_differences, test_gradient_rows_sum_to_zero, test_brute_force_loops]
     failed = 0
     for pin in pins:
         try:
@@ -329,3 +348,64 @@ def test_pins_catch_planted_mistakes(monkeypatch, name, fn):
         except AssertionError:
             failed += 1
     assert failed >= 1
+
+
+def _brute_force(H, W, idx, logit, mask):
+    """The definition written out with Python floats and loops only (no NumPy, no
+    BLAS): per token, z = H_t . W_v for every v, lse, p = softmax of the cached
+    logits (-inf -> 0), P = p pooled per id, l_t = sum_k p_k log P_{id_k} -
+    sum_k p_k z_{id_k} + M lse; loss = mean over unmasked tokens; G = (mask/N)(M
+    softmax(z) - P); dH = G W; dW = G^T H."""
+    import math
+    T, d, V, K = len(H), len(H[0]), len(W), len(idx[0])
+    N = sum(1 for t in range(T) if mask[t])
+    loss, ell, lse_all = 0.0, [], []
+    dH = [[0.0] * d for _ in range(T)]
+    dW = [[0.0] * d for _ in range(V)]
+    for t in range(T):
+        z = [sum(H[t][j] * W[v][j] for j in range(d)) for v in range(V)]
+        m = max(z)
+        lse = m + math.log(sum(math.exp(zv - m) for zv in z))
+        lm = max(logit[t])
+        if lm == -math.inf:
+            p = [0.0] * K
+        else:
+            e = [0.0 if l == -math.inf else math.exp(l - lm) for l in logit[t]]
+            p = [x / sum(e) for x in e]
+        P = {}
+        for k in range(K):
+            P[idx[t][k]] = P.get(idx[t][k], 0.0) + p[k]
+        M = sum(p)
+        l_t = sum(p[k] * math.log(P[idx[t][k]]) for k in range(K) if p[k] > 0)
+        l_t -= sum(p[k] * z[idx[t][k]] for k in range(K))
+        l_t += M * lse
+        ell.append(l_t)
+        lse_all.append(lse)
+        s = (1.0 / N) if (mask[t] and N) else 0.0
+        loss += s * l_t
+        for v in range(V):
+            g = s * (M * math.exp(z[v] - lse) - P.get(v, 0.0))
+            for j in range(d):
+                dH[t][j] += g * W[v][j]
+                dW[v][j] += g * H[t][j]
+    return loss, ell, lse_all, dH, dW
+
+
+def test_brute_force_loops():
+    rng = np.random.default_rng(97)
+    T, d, V, K = 5, 3, 7, 4
+    H = rng.standard_normal((T, d))
+    W = rng.standard_normal((V, d)) * 0.7
+    idx = rng.integers(0, V, (T, K)).astype(np.int32)
+    idx[1, 3] = idx[1, 0]            # a repeated id
+    logit = rng.standard_normal((T, K)) * 1.5
+    logit[2, 1] = -np.inf            # a dropped entry
+    mask = np.array([1, 1, 0, 1, 1], dtype=np.uint8)
+    bl, bell, blse, bdH, bdW = _brute_force(H.tolist(), W.tolist(), idx.tolist(),
+                                            logit.tolist(), mask.tolist())
+    r = oracle.fwd_bwd(H, W, idx, logit, mask)
+    assert abs(r["loss"] - bl) <= 1e-12 * max(1.0, abs(bl))
+    np.testing.assert_allclose(r["ell"], bell, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(r["lse"], blse, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(r["dH"], bdH, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(r["dW"], bdW, rtol=1e-11, atol=1e-13)
