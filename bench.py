@@ -165,27 +165,59 @@ def bus_id_of(dev: int) -> str:
     return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
 
 
-def oracle_rate(x, w, target_s: float, steps: int = 1):
-    """Time the fp64 oracle on a sample of the workload's tokens; tokens/s per step."""
+# Row counts of the two oracle calls each CPU-baseline step times (same in both legs).
+ORACLE_ROWS = (64, 192)
+
+
+def oracle_rate(x, w, steps: int = 1, warmup: int = 1):
+    """Per-token rate of the fp64 oracle on the host cores, from the slope of two calls.
+
+    W is widened to float64 once, before any timed call, so that no call pays the
+    multi-GB conversion (the oracle then uses the array as it is). Every step times
+    `oracle.sampled_rows` (lse, l_t, dH row and dW share of each sampled token) on
+    ORACLE_ROWS[0] and on ORACLE_ROWS[1] consecutive tokens of the workload; the
+    difference of the two times over the difference of the row counts is the
+    oracle's time per token, free of the per-call fixed costs (passes over W, the
+    V x d dW allocation). Returns (tokens/s of each timed step, per-call fixed
+    seconds of each step, row counts, cores).
+    """
     import oracle
     import threadpoolctl
-    rng_rows = np.arange(w.T)
     info = threadpoolctl.threadpool_info()
     cores = max([i.get("num_threads", 1) for i in info] + [1])
-    n0 = 8
-    for _ in range(2):  # the first call also pays one-time allocation costs
-        t0 = time.perf_counter()
-        oracle.sampled_rows(x["H"], x["W"], x["idx"], x["logit"], rng_rows[:n0], x["mask"],
-                            with_dW=True)
-        t_probe = time.perf_counter() - t0
-    n = int(min(4096, max(n0, n0 * target_s / max(t_probe, 1e-3))))
-    rates = []
-    for s in range(steps):
-        rows = rng_rows[(s * n) % w.T:][:n]
-        t0 = time.perf_counter()
-        oracle.sampled_rows(x["H"], x["W"], x["idx"], x["logit"], rows, x["mask"], with_dW=True)
-        rates.append(len(rows) / (time.perf_counter() - t0))
-    return rates, n, cores
+    W64 = np.asarray(x["W"], dtype=np.float64)  # untimed, once
+    n_a, n_b = ORACLE_ROWS
+    rates, fixed = [], []
+    for s in range(warmup + steps):
+        t_call = []
+        for n in (n_a, n_b):
+            start = (s * n_b) % max(1, w.T - n_b)
+            rows = np.arange(start, start + n)
+            t0 = time.perf_counter()
+            oracle.sampled_rows(x["H"], W64, x["idx"], x["logit"], rows, x["mask"], with_dW=True)
+            t_call.append(time.perf_counter() - t0)
+        per_tok = max(t_call[1] - t_call[0], 1e-9) / (n_b - n_a)
+        if s >= warmup:
+            rates.append(1.0 / per_tok)
+            fixed.append(t_call[0] - n_a * per_tok)
+    return rates, fixed, (n_a, n_b), cores
+
+
+def oracle_sample_text(rows, steps, fixed):
+    return (f"slope of two oracle calls per step ({rows[0]} and {rows[1]} consecutive tokens of the "
+            f"workload; full per-token path: lse, l_t, dH row, dW share; fp64 numpy/BLAS, W widened "
+            f"to fp64 once before timing), {steps} timed step(s); per-call fixed cost "
+            f"{statistics.median(fixed):.2f} s excluded")
+
+
+def bench_config(w, mask, chunk, recompute, world):
+    """The workload description of the bench line (the same for both arms)."""
+    return {"workload": w.name, "T": w.T, "d": w.d, "V": w.V, "K": w.K, "chunk": chunk,
+            "valid_tokens": int(w.T if mask is None else int(mask.astype(bool).sum())),
+            "backward": ("recompute logits" if recompute or w.dtype != "bf16"
+                         else "stored exp(z), bf16"),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "no flush: inputs larger than L2 (W alone is 1.16 GB)"}
 
 
 def run_reference(args, w, rank, world):
@@ -193,20 +225,17 @@ def run_reference(args, w, rank, world):
         return
     from chunked_kl_loss_logits_b200.workloads import make_inputs
     x = make_inputs(w)
-    per_step = 4.0
-    rates, n, cores = oracle_rate(x, w, per_step, steps=args.warmup + args.steps)
-    timed = rates[args.warmup:]
-    value = float(len(timed) / sum(1.0 / r for r in timed))  # tokens/s over the timed steps
-    ms = 1000.0 * n / value
+    rates, fixed, rows, cores = oracle_rate(x, w, steps=args.steps, warmup=args.warmup)
+    value = float(len(rates) / sum(1.0 / r for r in rates))  # tokens/s over the timed steps
+    ms = 1000.0 * (rows[1] - rows[0]) / value
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "T": w.T, "d": w.d, "V": w.V, "K": w.K, "chunk": w.chunk,
-                   "step": f"{n} tokens of the workload per step (whole per-token path incl. dW share)"},
+        "config": bench_config(w, x["mask"], args.chunk or w.chunk, args.recompute, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{n} tokens per step, {args.steps} timed steps"},
+                         "sample": oracle_sample_text(rows, args.steps, fixed)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -309,12 +338,24 @@ def run_ours(args, w, rank, world, local_rank):
     barrier()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev)
 
+    # the pages' two other loss forms beside this library, on this step's inputs
+    # (rank 0 at N = 1; the library's own buffers are released first)
+    compare = None
+    if rank == 0 and world == 1 and not args.no_compare and w.dtype == "bf16" and mask is None:
+        del out, ws, stag, Hh, ih, lh, mh
+        h.close()
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+        free, _ = torch.cuda.mem_get_info(dev)
+        compare = [{k: v for k, v in r.items() if k not in ("kind", "workload", "V", "d", "K")}
+                   for r in compare_forms(w, w.T, H, W, idx, logit, chunk, 2, dev, 0.92 * free)]
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rates, n, cores = oracle_rate(x, w, target_s=15.0)
-        cpu = {"value": rates[0], "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n} of the workload's {w.T} tokens, full per-token path "
-                         f"(lse, loss, dH row, dW share), fp64 numpy/BLAS"}
+        rates, fixed, rows, cores = oracle_rate(x, w, steps=2, warmup=1)
+        cpu = {"value": float(len(rates) / sum(1.0 / r for r in rates)), "unit": "tokens/s",
+               "cores": cores, "kind": "oracle",
+               "sample": oracle_sample_text(rows, len(rates), fixed)}
     if rank != 0:
         return
 
@@ -354,12 +395,7 @@ def run_ours(args, w, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": {"workload": w.name, "T": w.T, "d": w.d, "V": w.V, "K": w.K, "chunk": chunk,
-                   "valid_tokens": int(w.T if x["mask"] is None else int(x["mask"].astype(bool).sum())),
-                   "backward": ("recompute logits" if args.recompute or w.dtype != "bf16"
-                                else "stored exp(z), bf16"),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "no flush: inputs larger than L2 (W alone is 1.16 GB)"},
+        "config": bench_config(w, x["mask"], chunk, args.recompute, world),
         "tflops_useful": useful / (step_ms / 1e3) / 1e12,
         "tflops_executed": executed / (step_ms / 1e3) / 1e12,
         "frac_peak_useful": useful / (step_ms / 1e3) / 1e12 / pk_burst,
@@ -371,6 +407,7 @@ def run_ours(args, w, rank, world, local_rank):
         "e2e": {"value": job_tokens_per_s(w.T, world, args.steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
         "gpu_launches": launches,
+        "compare": compare,
         "clocks": clocks,
         "kernels": [{"name": s["name"], "launches": s["launches"],
                      "ms_per_step": s["total_ms"] / args.steps,
@@ -478,19 +515,82 @@ def _forward_chunked_kl(H, W, idx, logit, chunk):
     return total / H.shape[0]
 
 
+def compare_forms(w, T, H0, W0, idx, lg, chunk, steps, dev, budget):
+    """One sequence length: the pages' two other loss forms and this library on the same inputs.
+
+    Returns one record per method: peak device memory above the inputs and mean
+    forward + backward time over `steps` steps (CUDA events, after one untimed
+    step). A form whose estimated footprint exceeds `budget` bytes is not run
+    (reported as skipped); an out-of-memory exception is reported, not raised.
+    """
+    import torch
+
+    from chunked_kl_loss_logits_b200 import ckl
+    # bytes per T x V element held at the peak, as measured at 4K-32K tokens
+    # (dense: bf16 z and its grad plus ~4 fp32 T x V tensors; forward-chunked: bf16 z,
+    # its grad and one fp32 chunk copy), with a margin
+    est = {"dense_kl": T * w.V * 23, "forward_chunked": T * w.V * 8.5, "ckl": 0}
+    recs = []
+    for method in ("dense_kl", "forward_chunked", "ckl"):
+        rec = {"kind": "compare", "method": method, "workload": w.name, "T": T, "V": w.V,
+               "d": w.d, "K": w.K, "chunk": chunk if method != "dense_kl" else None}
+        if est[method] > budget:
+            rec["status"] = "skipped: estimated %.0f GiB above the %.0f GiB budget" % (
+                est[method] / 2**30, budget / 2**30)
+            recs.append(rec)
+            continue
+        H = H0.detach().clone().requires_grad_(method != "ckl")
+        W = W0.detach().clone().requires_grad_(method != "ckl")
+        h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=chunk, device=dev) if method == "ckl" else None
+
+        def step():
+            if method == "ckl":
+                return h.fwd_bwd(H, W, idx, lg, None, chunk=chunk, sync=False)[0]
+            H.grad = W.grad = None
+            loss = _dense_kl(H, W, idx, lg) if method == "dense_kl" else \
+                _forward_chunked_kl(H, W, idx, lg, chunk)
+            loss.backward()
+            return loss.detach()
+
+        try:
+            torch.cuda.synchronize(dev)
+            torch.cuda.empty_cache()
+            base = torch.cuda.memory_allocated(dev)
+            torch.cuda.reset_peak_memory_stats(dev)
+            loss = step()
+            torch.cuda.synchronize(dev)
+            peak = torch.cuda.max_memory_allocated(dev) - base
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                loss = step()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1) / steps
+            rec.update(status="ok", loss=float(loss), peak_gib_above_inputs=peak / 2**30,
+                       ms_per_step=ms, tokens_per_s=T / (ms / 1e3),
+                       tflops_useful=6.0 * T * w.V * w.d / (ms / 1e3) / 1e12)
+        except torch.cuda.OutOfMemoryError as e:
+            rec["status"] = "out of memory: " + str(e).splitlines()[0][:120]
+        recs.append(rec)
+        del H, W
+        if h is not None:
+            h.close()
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+    return recs
+
+
 def run_compare(args, w):
     """The pages' two other loss forms, in plain PyTorch on this GPU, beside this library.
 
     For T in a range of sequence lengths on the workload's (V, d, K): peak device
     memory above the inputs and mean forward + backward time of each form, one JSON
-    line per (method, T). A form whose estimated footprint exceeds the memory
-    budget is not run (reported as skipped); an out-of-memory exception is
-    reported, not raised. Inputs are the workload's own (distinct teacher ids, so
+    line per (method, T). Inputs are the workload's own (distinct teacher ids, so
     the dense scatter and the sparse forms agree).
     """
     import torch
 
-    from chunked_kl_loss_logits_b200 import ckl
     from chunked_kl_loss_logits_b200.workloads import make_inputs
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -504,58 +604,8 @@ def run_compare(args, w):
         idx = torch.from_numpy(x["idx"]).to(dev)
         lg = torch.from_numpy(x["logit"]).to(dev)
         del x
-        # bytes per T x V element held at the peak, as measured at 4K-32K tokens
-        # (dense: bf16 z and its grad plus ~4 fp32 T x V tensors; forward-chunked: bf16 z,
-        # its grad and one fp32 chunk copy), with a margin
-        est = {"dense_kl": T * w.V * 23, "forward_chunked": T * w.V * 8.5, "ckl": 0}
-        for method in ("dense_kl", "forward_chunked", "ckl"):
-            rec = {"kind": "compare", "method": method, "workload": w.name, "T": T, "V": w.V,
-                   "d": w.d, "K": w.K, "chunk": chunk if method != "dense_kl" else None}
-            if est[method] > budget:
-                rec["status"] = "skipped: estimated %.0f GiB above the %.0f GiB budget" % (
-                    est[method] / 2**30, budget / 2**30)
-                print(json.dumps(rec), flush=True)
-                continue
-            H = H0.clone().requires_grad_(method != "ckl")
-            W = W0.clone().requires_grad_(method != "ckl")
-            h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=chunk, device=dev) if method == "ckl" else None
-
-            def step():
-                if method == "ckl":
-                    return h.fwd_bwd(H, W, idx, lg, None, chunk=chunk, sync=False)[0]
-                H.grad = W.grad = None
-                loss = _dense_kl(H, W, idx, lg) if method == "dense_kl" else \
-                    _forward_chunked_kl(H, W, idx, lg, chunk)
-                loss.backward()
-                return loss.detach()
-
-            try:
-                torch.cuda.synchronize(dev)
-                torch.cuda.empty_cache()
-                base = torch.cuda.memory_allocated(dev)
-                torch.cuda.reset_peak_memory_stats(dev)
-                loss = step()
-                torch.cuda.synchronize(dev)
-                peak = torch.cuda.max_memory_allocated(dev) - base
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                n = args.compare_steps
-                e0.record()
-                for _ in range(n):
-                    loss = step()
-                e1.record()
-                torch.cuda.synchronize(dev)
-                ms = e0.elapsed_time(e1) / n
-                rec.update(status="ok", loss=float(loss), peak_gib_above_inputs=peak / 2**30,
-                           ms_per_step=ms, tokens_per_s=T / (ms / 1e3),
-                           tflops_useful=6.0 * T * w.V * w.d / (ms / 1e3) / 1e12)
-            except torch.cuda.OutOfMemoryError as e:
-                rec["status"] = "out of memory: " + str(e).splitlines()[0][:120]
+        for rec in compare_forms(w, T, H0, W0, idx, lg, chunk, args.compare_steps, dev, budget):
             print(json.dumps(rec), flush=True)
-            del H, W
-            if h is not None:
-                h.close()
-            torch.cuda.synchronize(dev)
-            torch.cuda.empty_cache()
         del H0, W0, idx, lg
 
 
@@ -685,6 +735,8 @@ def main():
     ap.add_argument("--workload", default="bf16_32k")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-compare", action="store_true",
+                    help="skip the pages' two other loss forms on this workload's inputs (N = 1)")
     ap.add_argument("--sweep", action="store_true",
                     help="256K workload: throughput vs chunk and peak memory vs T (extra JSON lines)")
     ap.add_argument("--sweep-steps", type=int, default=3)

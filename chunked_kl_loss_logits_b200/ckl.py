@@ -468,48 +468,85 @@ class ChunkedKL:
 
 class _ChunkedKLFn(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, H, W, idx, logit, mask, handle, chunk):
+    def forward(ctx, H, W, idx, logit, mask, handle, chunk, check):
         loss, dH, dW = handle.fwd_bwd(H.detach(), W.detach(), idx, logit, mask, chunk=chunk,
                                       sync=False)
         ctx.save_for_backward(dH, dW)
         ctx.w_dtype = W.dtype
+        ctx.handle, ctx.check = handle, check
         return loss
 
     @staticmethod
     def backward(ctx, g):
-        dH, dW = ctx.saved_tensors
-        return (dH * g.to(dH.dtype), (dW * g).to(ctx.w_dtype), None, None, None, None, None)
-
-
-class _VocabParallelKLFn(torch.autograd.Function):
-    @staticmethod
-    def forward(ctx, H, W_shard, idx, logit, mask, handle, chunk, group):
-        loss, dH, dW = handle.fwd_bwd_vocab_parallel(group, H.detach(), W_shard.detach(), idx,
-                                                     logit, mask, chunk=chunk, sync=False)
-        ctx.save_for_backward(dH, dW)
-        ctx.w_dtype = W_shard.dtype
-        return loss
-
-    @staticmethod
-    def backward(ctx, g):
+        if ctx.check:
+            ctx.handle.sync_status()  # raises CKLError on a device-detected error
         dH, dW = ctx.saved_tensors
         return (dH * g.to(dH.dtype), (dW * g).to(ctx.w_dtype), None, None, None, None, None, None)
 
 
+class _VocabParallelKLFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, H, W_shard, idx, logit, mask, handle, chunk, group, check):
+        loss, dH, dW = handle.fwd_bwd_vocab_parallel(group, H.detach(), W_shard.detach(), idx,
+                                                     logit, mask, chunk=chunk, sync=False)
+        ctx.save_for_backward(dH, dW)
+        ctx.w_dtype = W_shard.dtype
+        ctx.handle, ctx.check = handle, check
+        return loss
+
+    @staticmethod
+    def backward(ctx, g):
+        if ctx.check:
+            ctx.handle.sync_status()
+        dH, dW = ctx.saved_tensors
+        return (dH * g.to(dH.dtype), (dW * g).to(ctx.w_dtype), None, None, None, None, None, None,
+                None)
+
+
+_HANDLES = {}
+
+
+def handle_for(W, K: int, chunk: int | None = None) -> ChunkedKL:
+    """The cached handle for W's device, dtype and shape with K cached entries.
+
+    chunked_kl_loss calls this when it is given no handle, so a training loop
+    creates one handle per LM-head shape (ckl_create allocates and synchronises
+    the device) instead of one per step. The handle is replaced by one with a
+    larger max_chunk when a call asks for a chunk above the cached one's.
+    """
+    dev = W.device
+    key = (dev.type, dev.index, W.dtype, W.shape[0], W.shape[1], K)
+    h = _HANDLES.get(key)
+    need = max(chunk or 4096, 1)
+    if h is None or h.max_chunk < need:
+        if h is not None:
+            h.close()
+        h = ChunkedKL(W.shape[0], W.shape[1], K, dtype=W.dtype, max_chunk=need, device=dev)
+        _HANDLES[key] = h
+    return h
+
+
 def chunked_kl_loss(H, W, idx, logit, mask=None, chunk=None, handle: ChunkedKL | None = None,
-                    group: VocabGroup | None = None):
+                    group: VocabGroup | None = None, check: bool = True):
     """Autograd-friendly mean top-K forward KL; the gradients come from the fused call.
 
     With `group`, W is this rank's vocabulary rows (vocab_shards) and the loss is the
     full-vocabulary one, identical on every rank; H's gradient is the full dH on
-    every rank and W's is this rank's rows.
+    every rank and W's is this rank's rows. Without `handle` the handle cached for
+    W's shape (handle_for) is used.
+
+    check=True: backward() waits for the call's stream and raises CKLError if the
+    device reported an error (a teacher id outside [0, V), a pipeline timeout);
+    the outputs of such a call are undefined. check=False: nothing waits; the
+    device status stays set in the handle (errors of later calls add to it) until
+    the caller reads it with handle.sync_status() (handle_for(W, K) gives the
+    cached handle), which raises and clears it.
     """
     if handle is None:
-        handle = ChunkedKL(W.shape[0], W.shape[1], idx.shape[1], dtype=W.dtype,
-                           max_chunk=max(chunk or 4096, 1), device=W.device)
+        handle = handle_for(W, idx.shape[1], chunk)
     if group is not None:
-        return _VocabParallelKLFn.apply(H, W, idx, logit, mask, handle, chunk, group)
-    return _ChunkedKLFn.apply(H, W, idx, logit, mask, handle, chunk)
+        return _VocabParallelKLFn.apply(H, W, idx, logit, mask, handle, chunk, group, check)
+    return _ChunkedKLFn.apply(H, W, idx, logit, mask, handle, chunk, check)
 
 
 def forward_static(H, W, idx, logit, mask=None, chunk: int = 2048, stream=None,

@@ -1028,7 +1028,8 @@ StaticDevice g_static_dev[kStaticMaxDevices];
 
 // Once per device, with that device current: the device address of the static
 // array (the host-side symbol is only a stand-in), the SM count and the TMA
-// descriptor encoder.
+// descriptor encoder. The address belongs to the device's current CUDA context;
+// a cudaDeviceReset would end that context, which the header rules out.
 ckl_status static_setup(int device, StaticDevice** out) {
   std::lock_guard<std::mutex> lock(g_static_mu);
   StaticDevice& sd = g_static_dev[device];
@@ -1065,6 +1066,8 @@ extern "C" ckl_status ckl_forward_static(int device, ckl_dtype dtype, int64_t V,
   if (dtype != CKL_F32 && dtype != CKL_BF16) return CKL_ERR_INVALID_ARG;
   if (V < 1 || d < 1 || K < 1 || chunk < 1 || T < 0 || device < 0 || device >= kStaticMaxDevices)
     return CKL_ERR_INVALID_ARG;
+  // Without a handle the device status can only be returned by this call itself.
+  if (!loss_host) return CKL_ERR_INVALID_ARG;
   if (d % 8 != 0 || K > 1024 || V > (int64_t)INT32_MAX / 2 || d > 65536 || chunk > INT32_MAX)
     return CKL_ERR_UNSUPPORTED;
   const int64_t per_warp =
@@ -1095,7 +1098,7 @@ extern "C" ckl_status ckl_forward_static(int device, ckl_dtype dtype, int64_t V,
   st = run(&c, H, W, topk_idx, topk_logit, mask, T, chunk, loss, nullptr, nullptr, token_lse,
            token_loss, sd->scratch + kStaticStatusBytes, kStaticScratchBytes - kStaticStatusBytes,
            s, false);
-  if (st != CKL_OK || !loss_host) return st;
+  if (st != CKL_OK) return st;
   unsigned dev_status = 0;
   float host_loss = 0.f;
   if (cudaMemcpyAsync(&host_loss, loss, sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess ||

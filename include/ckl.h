@@ -151,7 +151,14 @@ ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t
  * streams or host threads) race on the array and must not be issued.
  * Arguments are those of ckl_create (device, dtype, V, d, K) followed by those
  * of ckl_forward without the workspace; chunk has no max_chunk bound other than
- * the scratch size. loss_host: as in ckl_forward (pageable memory is fine). */
+ * the scratch size. loss_host is required (NULL gives CKL_ERR_INVALID_ARG): with
+ * no handle there is no later ckl_sync_status, and the next call clears the
+ * shared status word, so every call waits for its stream, stores the loss in
+ * *loss_host (pageable memory is fine) and returns the device-detected status
+ * (CKL_ERR_INDEX_RANGE for a teacher id outside [0, V), ...).
+ * The cached device address of the array stays valid for the life of the
+ * process's CUDA context on that device: after cudaDeviceReset on a device this
+ * entry point must not be called on it again in the same process. */
 ckl_status ckl_forward_static(int device, ckl_dtype dtype, int64_t V, int64_t d, int64_t K,
                               const void* H, const void* W, const int32_t* topk_idx,
                               const float* topk_logit, const uint8_t* mask, int64_t T,

@@ -10,6 +10,23 @@ def rel_fro(a, b) -> float:
     return float(np.linalg.norm(a - b) / nb) if nb > 0 else float(np.linalg.norm(a))
 
 
+def worst_row(a, b) -> float:
+    """Largest per-row relative error max_r |a_r - b_r| / |b_r| (Frobenius norms of rows).
+
+    A row where b is exactly zero counts as 0 if a is zero there too, else as inf,
+    so a defect confined to a few rows or one tile cannot hide under a whole-tensor
+    norm.
+    """
+    a = np.asarray(a, np.float64).reshape(len(a), -1)
+    b = np.asarray(b, np.float64).reshape(len(b), -1)
+    nb = np.linalg.norm(b, axis=1)
+    na = np.linalg.norm(a - b, axis=1)
+    zero = nb == 0
+    if np.any(zero & (na > 0)):
+        return float("inf")
+    return float(np.max(na[~zero] / nb[~zero])) if np.any(~zero) else 0.0
+
+
 def rel(a, b) -> float:
     return abs(float(a) - float(b)) / max(abs(float(b)), 1e-30)
 
@@ -35,4 +52,13 @@ def f64(t):
 TOL = {
     "f32": {"loss": 1e-5, "grad": 1e-4},
     "bf16": {"loss": 1e-3, "grad": 2e-2},
+}
+
+# Worst single row (a token's dH row, a vocabulary id's dW row) and worst single
+# token (absolute error of lse_t and l_t, in nats). Rounding spreads evenly over
+# rows, so these sit a few times above the whole-tensor errors; a wrong tile or a
+# wrong token shows up as an error of order one.
+ROW_TOL = {
+    "f32": {"grad_row": 1e-3, "tok_abs": 1e-4},
+    "bf16": {"grad_row": 5e-2, "tok_abs": 2e-3},
 }

@@ -12,7 +12,7 @@ import torch
 import oracle
 from chunked_kl_loss_logits_b200 import ckl
 from chunked_kl_loss_logits_b200.workloads import WORKLOADS, make_inputs, small_case
-from tests._helpers import TOL, f64, rel, rel_fro, upload
+from tests._helpers import ROW_TOL, TOL, f64, rel, rel_fro, upload, worst_row
 
 pytestmark = pytest.mark.gpu
 
@@ -35,13 +35,22 @@ def run_and_compare(x, dt, chunk, tol=None, strict=None, recompute=False):
         "dW": rel_fro(f64(dW), r["dW"]),
         "lse": rel_fro(f64(lse), r["lse"]),
         "ell": rel_fro(f64(ell), r["ell"]),
+        "dH_row": worst_row(f64(dH), r["dH"]),
+        "dW_row": worst_row(f64(dW), r["dW"]),
+        "lse_tok": float(np.max(np.abs(f64(lse) - r["lse"]), initial=0.0)),
+        "ell_tok": float(np.max(np.abs(f64(ell) - r["ell"]), initial=0.0)),
     }
+    row_tol = ROW_TOL[dt]
     print(dt, "recompute" if recompute else "stored", x["H"].shape, V, K, chunk,
           {k: f"{v:.2e}" for k, v in errs.items()})
     assert errs["loss"] <= tol["loss"], errs
     assert errs["dH"] <= tol["grad"], errs
     assert errs["dW"] <= tol["grad"], errs
     assert errs["lse"] <= tol["loss"], errs
+    assert errs["dH_row"] <= row_tol["grad_row"], errs
+    assert errs["dW_row"] <= row_tol["grad_row"], errs
+    assert errs["lse_tok"] <= row_tol["tok_abs"], errs
+    assert errs["ell_tok"] <= row_tol["tok_abs"], errs
     if strict:
         for k, bound in strict.items():
             assert errs[k] <= bound, (k, errs)
@@ -239,6 +248,40 @@ def test_autograd_function():
     assert loss.item() == l2.item()
     assert torch.equal(Hp.grad, dH * 2.0)
     assert torch.allclose(Wp.grad.float(), (dW * 2.0).to(torch.bfloat16).float())
+
+
+def test_autograd_training_steps_reuse_one_handle():
+    # two steps through the autograd wrapper with no handle: one cached handle,
+    # the launches of two fused calls on it, and a device error raised at backward
+    x = small_case(260, 64, 700, 8, seed=23, dtype="bf16", teacher_var=3.0, ids="zipf")
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    Wp = W.clone().requires_grad_(True)
+    h = ckl.handle_for(Wp, 8, 128)
+    n0 = h.launch_count()
+    for _ in range(2):
+        Hp = H.clone().requires_grad_(True)
+        loss = ckl.chunked_kl_loss(Hp, Wp, idx, logit, mask, chunk=128)
+        loss.backward()
+        assert ckl.handle_for(Wp, 8, 128) is h
+    # mask count + 3 chunks x 8 kernels + loss, per step
+    assert h.launch_count() - n0 == 2 * (1 + 3 * 8 + 1)
+    ref = ckl.ChunkedKL(700, 64, 8, max_chunk=128)
+    l1, dH1, dW1 = ref.fwd_bwd(H, W, idx, logit, mask, chunk=128)
+    assert loss.item() == l1.item() and torch.equal(Hp.grad, dH1)
+    ref.close()
+    bad = idx.clone()
+    bad[5, 2] = 700
+    Hp = H.clone().requires_grad_(True)
+    loss = ckl.chunked_kl_loss(Hp, Wp, bad, logit, mask, chunk=128)
+    with pytest.raises(ckl.CKLError) as e:
+        loss.backward()
+    assert e.value.code == 4
+    # check=False defers the report to the caller's own sync_status
+    Hp = H.clone().requires_grad_(True)
+    ckl.chunked_kl_loss(Hp, Wp, bad, logit, mask, chunk=128, check=False).backward()
+    with pytest.raises(ckl.CKLError):
+        h.sync_status()
+    h.sync_status()  # cleared
 
 
 def test_workspace_is_linear_in_tokens_and_bounded_by_chunk():

@@ -1,12 +1,17 @@
 """The allocation-free forward entry point (ckl_forward_static), called through
-the C ABI, against the existing ckl_forward on the same inputs.
+the C ABI, against the existing ckl_forward on the same inputs and against the
+fp64 oracle.
 
 Callers that may not call cudaMalloc (a host runtime that owns all device memory
 through its own allocator, a latency-critical loop that cannot take the
 device-wide synchronisation of an allocation) use this variant: its scratch is a
-fixed 32 MiB device array inside the library, shared by all calls. The test makes
-two calls in a row with different inputs, so state left in the shared array by
-the first call would show up in the second. This file is collected last.
+fixed 32 MiB device array inside the library, shared by all calls. Both entry
+points run the same launch sequence on the same inputs, so their outputs must be
+bit-identical. The test makes two calls in a row with different inputs, so state
+left in the shared array by the first call (partials, the status word) would
+show up in the second; an out-of-range teacher id must come back as a status
+through the shared status word and must not leak into the next call. This file
+is collected last.
 """
 import ctypes
 
@@ -14,13 +19,14 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from chunked_kl_loss_logits_b200 import build, ckl
 from chunked_kl_loss_logits_b200.workloads import small_case
-from tests._helpers import rel, rel_fro, upload
+from tests._helpers import TOL, f64, rel, rel_fro, upload
 
 pytestmark = pytest.mark.gpu
 
-TOL = {torch.bfloat16: 1e-3, torch.float32: 1e-5}
+DT = {torch.bfloat16: "bf16", torch.float32: "f32"}
 _P, _I64 = ctypes.c_void_p, ctypes.c_int64
 
 
@@ -33,7 +39,7 @@ def _entry():
     return f
 
 
-def _call_static(f, H, W, idx, logit, mask, chunk):
+def _call_static(f, H, W, idx, logit, mask, chunk, with_host=True):
     T, d = H.shape
     V, K = W.shape[0], idx.shape[1]
     loss = torch.empty((), dtype=torch.float32, device="cuda")
@@ -43,28 +49,63 @@ def _call_static(f, H, W, idx, logit, mask, chunk):
     p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
     code = f(torch.cuda.current_device(), 0 if H.dtype == torch.float32 else 1, V, d, K, p(H),
              p(W), p(idx), p(logit), p(mask), T, chunk, p(loss), p(lse), p(ell),
-             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream), ctypes.byref(host))
+             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream),
+             ctypes.byref(host) if with_host else None)
     return code, loss, lse, ell, host.value
+
+
+def _cases(dt):
+    return [(small_case(300, 128, 3000, 16, seed=31, dtype=dt, teacher_var=3.0, ids="zipf",
+                        packing=True), 128),
+            (small_case(517, 64, 1777, 12, seed=32, dtype=dt, teacher_var=3.0, ids="zipf"), 200)]
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_static_forward_matches_forward_twice(dtype):
     f = _entry()
-    dt = "bf16" if dtype == torch.bfloat16 else "f32"
-    cases = [small_case(300, 128, 3000, 16, seed=31, dtype=dt, teacher_var=3.0, ids="zipf",
-                        packing=True),
-             small_case(517, 64, 1777, 12, seed=32, dtype=dt, teacher_var=3.0, ids="zipf")]
-    for x, chunk in zip(cases, (128, 200)):
+    tol = TOL[DT[dtype]]
+    for x, chunk in _cases(DT[dtype]):
         H, W, idx, logit, mask = upload(x, dtype)
         code, loss, lse, ell, lh = _call_static(f, H, W, idx, logit, mask, chunk)
         assert code == 0, ckl.lib().ckl_status_str(code)
         h = ckl.ChunkedKL(W.shape[0], W.shape[1], idx.shape[1], dtype=dtype, max_chunk=chunk)
         l0, lse0, ell0 = h.forward(H, W, idx, logit, mask, chunk=chunk, token_stats=True)
-        assert lh == loss.item()
-        assert rel(loss.item(), l0.item()) <= TOL[dtype]
-        assert rel_fro(lse.double().cpu().numpy(), lse0.double().cpu().numpy()) <= TOL[dtype]
-        assert rel_fro(ell.double().cpu().numpy(), ell0.double().cpu().numpy()) <= TOL[dtype]
         h.close()
+        # same launch sequence on the same inputs: identical bits
+        assert lh == loss.item()
+        assert torch.equal(loss, l0) and torch.equal(lse, lse0) and torch.equal(ell, ell0)
+        # and the method's values, against the fp64 oracle
+        r = oracle.fwd_bwd(x["H"], x["W"], x["idx"], x["logit"], x["mask"])
+        assert rel(loss.item(), r["loss"]) <= tol["loss"]
+        assert rel_fro(f64(lse), r["lse"]) <= tol["loss"]
+        assert rel_fro(f64(ell), r["ell"]) <= tol["loss"]
+
+
+def test_static_forward_reports_a_bad_id_then_recovers():
+    f = _entry()
+    (x, chunk), (y, chunk2) = _cases("bf16")
+    bad = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in x.items()}
+    bad["idx"][7, 3] = 3000    # = V: outside [0, V)
+    H, W, idx, logit, mask = upload(bad, torch.bfloat16)
+    code, *_ = _call_static(f, H, W, idx, logit, mask, chunk)
+    assert code == 4, ckl.lib().ckl_status_str(code)        # CKL_ERR_INDEX_RANGE
+    # the next call starts from a cleared status word and gives the exact result
+    H, W, idx, logit, mask = upload(y, torch.bfloat16)
+    code, loss, lse, ell, lh = _call_static(f, H, W, idx, logit, mask, chunk2)
+    assert code == 0, ckl.lib().ckl_status_str(code)
+    h = ckl.ChunkedKL(W.shape[0], W.shape[1], idx.shape[1], max_chunk=chunk2)
+    l0, lse0, ell0 = h.forward(H, W, idx, logit, mask, chunk=chunk2, token_stats=True)
+    h.close()
+    assert torch.equal(loss, l0) and torch.equal(lse, lse0) and torch.equal(ell, ell0)
+
+
+def test_static_forward_needs_loss_host():
+    # without a handle the status can only come back from the call itself
+    f = _entry()
+    x, chunk = _cases("bf16")[0]
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    code, *_ = _call_static(f, H, W, idx, logit, mask, chunk, with_host=False)
+    assert code == 1                                           # CKL_ERR_INVALID_ARG
 
 
 def test_static_forward_rejects_sizes_beyond_its_scratch():
