@@ -12,11 +12,13 @@
 //                                   sum p z over the ids in the tile (bf16); stored-exp
 //                                   mode also keeps e = exp(z - tile max) in bf16
 //     combine                       lse_t, l_t, gradient multipliers
-//     stored-exp mode:  scale_e     G = e * (mask/N) M exp(tile max - lse)       (in place)
+//     stored-exp mode:  repair      rows whose stored exps used a per-tile reference
+//                                   rescaled to the row's reference R (usually none)
 //     recompute mode:   GRAD        G = (mask/N) M exp(z - lse), z formed again
-//     fixup                         G at the K ids: subtract (mask/N) P, in place
-//     DH contraction (+ reduce)     dH_c = G W
-//     DW contraction                dW (+)= G^T H_c   (TMA reduce-add into dW)
+//     fixup                         G at the K ids: subtract (mask/N) P (stored-exp mode:
+//                                   P / (M exp(R - lse)), as G = c_t E there), in place
+//     DH contraction (+ reduce)     dH_c = G W (stored-exp: c_t (E W), and Hs = c_t H_c)
+//     DW contraction                dW (+)= G^T H_c   (stored-exp: E^T Hs; TMA reduce-add)
 //   loss_finalize                   loss = sum mask l / N
 // The gradient buffer G is the only one that grows with V, and it is bounded by
 // chunk x V; everything else is O(T) or O(chunk x K).
@@ -54,7 +56,7 @@ enum KernelId {
   KID_VP_MERGE, KID_DH_F32, KID_TO_BF16, KID_VP_GATHER, KID_VP_REDUCE, KID_COUNT
 };
 const char* kKernelNames[KID_COUNT] = {"mask_count", "teacher_topk", "lse_gemm", "lse_combine",
-                                       "grad_gemm", "scale_e", "topk_fixup", "dh_gemm",
+                                       "grad_gemm", "row_repair", "topk_fixup", "dh_gemm",
                                        "dh_reduce", "dw_gemm", "loss_finalize", "cache_max_gemm",
                                        "cache_threshold", "cache_emit_gemm", "cache_select",
                                        "vp_merge", "dh_reduce_f32", "dh_to_bf16",
@@ -108,7 +110,7 @@ struct WsPlan {
   int n_split = 1; // dH contraction splits (bf16)
   size_t off_ell = 0, off_lse = 0, off_misc = 0, off_tok = 0, off_cst = 0, off_zk = 0,
          off_Pk = 0, off_part = 0, off_xpart = 0, off_sid = 0, off_sp = 0, off_G = 0, off_dHp = 0,
-         total = 0;
+         off_rep = 0, off_Hs = 0, total = 0;
   // vocabulary split over ranks: this rank's stats, the gathered stats, dH_c in fp32
   size_t off_stats = 0, off_stats_all = 0, off_dhf = 0;
 };
@@ -158,7 +160,12 @@ WsPlan plan(const ckl_ctx* h, int64_t T, int64_t chunk, bool backward, int world
     // bf16: blocked, 64 x 64 element blocks (8 KB); fp32: row-major, ldG
     p.off_G = bf16 ? take((size_t)((p.Tc + 63) / 64) * ((h->V + 63) / 64) * 8192)
                    : take((size_t)p.Tc * p.ldG * 4);
-    if (bf16) p.off_dHp = take((size_t)p.n_split * p.Tc * h->d * 4);
+    if (bf16) {
+      p.off_dHp = take((size_t)p.n_split * p.Tc * h->d * 4);
+      // stored-exp backward: the repair list (count, rows) and the scaled H_c of DW
+      p.off_rep = take((size_t)(p.Tc + 1) * 4);
+      p.off_Hs = take((size_t)p.Tc * h->d * 2);
+    }
   }
   if (world > 0) {
     p.off_stats = take((size_t)p.Tc * 16);
@@ -301,6 +308,9 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
   b.sp = h->dtype == CKL_BF16 ? reinterpret_cast<float*>(base + P.off_sp) : nullptr;
   b.G = backward ? base + P.off_G : nullptr;
   b.dHp = (backward && h->dtype == CKL_BF16) ? reinterpret_cast<float*>(base + P.off_dHp) : nullptr;
+  b.rep = (backward && h->dtype == CKL_BF16) ? reinterpret_cast<int*>(base + P.off_rep) : nullptr;
+  uint16_t* Hs = (backward && h->dtype == CKL_BF16) ? reinterpret_cast<uint16_t*>(base + P.off_Hs)
+                                                     : nullptr;
   float* ell_all = reinterpret_cast<float*>(base + P.off_ell);
   float* lse_all = reinterpret_cast<float*>(base + P.off_lse);
   float4* stats = group ? reinterpret_cast<float4*>(base + P.off_stats) : nullptr;
@@ -357,9 +367,13 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     }
     if (ready) chk(cudaStreamWaitEvent(s, ready[t0 / chunk], 0));
 
+    // bf16 backward keeps the exps of the forward contraction (unless recomputing)
+    const bool store_e = bf16 && backward && !h->recompute;
     if (bf16) {
-      chk(L(KID_GATHER, 0, (double)Tc * K * 16.0, [&] {
-        launch_teacher(idx, logit, t0, Tc, V_all, v0, K, b, h->d_status, s);
+      chk(L(KID_GATHER, 0, (double)Tc * K * 16.0 + (store_e ? 4.0 * Tc * d : 0.0), [&] {
+        launch_teacher(idx, logit, t0, Tc, V_all, v0, V, K, b, h->d_status,
+                       store_e ? reinterpret_cast<const uint16_t*>(Hc) : nullptr,
+                       static_cast<const uint16_t*>(W), d, s);
       }));
     } else {
       chk(L(KID_GATHER, 2.0 * Tc * K * d, (double)Tc * (K * 8.0 + d * esz + K * d * esz), [&] {
@@ -369,8 +383,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     }
 
     // bf16: z = H_c W^T on the tensor cores. Stored-exp mode also writes
-    // e = exp(z - tile max) into the gradient buffer (map c) for the backward.
-    const bool store_e = bf16 && backward && !h->recompute;
+    // exp(z - row reference) into the gradient buffer (map c) for the backward.
     TcMaps mz;
     if (bf16) {
       if (!make_map(h, &mz.a, Hc, d, Tc, (uint64_t)d * 2, 64, 128) ||
@@ -388,7 +401,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
         TcLaunch p{};
         p.kind = TcKind::LSE; p.M = Tc; p.N = V; p.n_kb = (d + 63) / 64; p.n_split = 1; p.V = V;
         p.part = b.part; p.part_ld = Tc; p.store_e = store_e ? 1 : 0;
-        p.sid = b.sid; p.sp = b.sp; p.xpart = b.xpart; p.K = K;
+        p.sid = b.sid; p.sp = b.sp; p.xpart = b.xpart; p.K = K; p.tok = b.tok;
         p.status = h->d_status; p.num_sms = h->num_sms;
         launch_tc(mz, p, s);
       } else {
@@ -397,20 +410,21 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
       }
     }));
     chk(L(KID_COMBINE, 0, (double)P.n_vt * Tc * 8, [&] {
-      launch_combine(t0, Tc, P.n_vt, mask, b, lse_all, ell_all, stats, s);
+      launch_combine(t0, Tc, P.n_vt, mask, b, lse_all, ell_all, stats, store_e, s);
     }));
     if (group) {
       // this rank's (max, sum, cross) per token to every rank; merged in rank order
       gather();
       chk(L(KID_VP_MERGE, 0, (double)Tc * (group->world * 16.0 + 24.0), [&] {
-        launch_vp_merge(t0, Tc, group->world, stats_all, mask, b, lse_all, ell_all, s);
+        launch_vp_merge(t0, Tc, group->world, group->rank, stats_all, mask, b, lse_all, ell_all,
+                        store_e, s);
       }));
     }
     if (!backward) continue;
 
     if (store_e) {
-      chk(L(KID_SCALE, 0, (double)Tc * V * 4, [&] {
-        launch_scale_e(static_cast<uint16_t*>(b.G), Tc, V, b, s);
+      chk(L(KID_SCALE, 0, 0, [&] {
+        launch_repair(static_cast<uint16_t*>(b.G), Tc, V, b, h->num_sms, s);
       }));
     } else {
       chk(L(KID_GRAD, zflops, (double)Tc * V * esz, [&] {
@@ -427,7 +441,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
       }));
     }
     chk(L(KID_FIXUP, 0, (double)Tc * K * (12.0 + 2 * esz), [&] {
-      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, v0, (V + 63) / 64, b, false, s);
+      if (bf16) launch_fixup<uint16_t>(idx, t0, Tc, K, V, v0, (V + 63) / 64, b, store_e, s);
       else launch_fixup<float>(idx, t0, Tc, K, V, v0, P.ldG, b, false, s);
     }));
 
@@ -437,7 +451,8 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
       if (!make_map_g(h, &mh.a, b.G, V, Tc, 64, 1, 2) ||
           !make_map(h, &mh.b, W, d, V, (uint64_t)d * 2, 64, 64) ||
           !make_map_g(h, &mw.a, b.G, V, Tc, 64, 2, 1) ||
-          !make_map(h, &mw.b, Hc, d, Tc, (uint64_t)d * 2, 64, 64) ||
+          !make_map(h, &mw.b, store_e ? static_cast<const void*>(Hs) : Hc, d, Tc,
+                    (uint64_t)d * 2, 64, 64) ||
           !make_map(h, &mw.c, dW, d, V, (uint64_t)d * 4, 32, 32, true)) {
         map_failed = true;
         if (!group) return CKL_ERR_CUDA;
@@ -452,14 +467,19 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
         launch_tc(mh, p, s);
       }));
       if (!group) {
-        chk(L(KID_DH_REDUCE, 0, (double)Tc * d * (4.0 * P.n_split + 2.0), [&] {
+        chk(L(KID_DH_REDUCE, 0, (double)Tc * d * (4.0 * P.n_split + 2.0 + (store_e ? 4.0 : 0.0)),
+              [&] {
           launch_dh_reduce_bf16(b.dHp, P.n_split, (int64_t)Tc * d,
-                                reinterpret_cast<uint16_t*>(dHc), s);
+                                reinterpret_cast<uint16_t*>(dHc), d, store_e ? b.cst : nullptr,
+                                reinterpret_cast<const uint16_t*>(Hc), store_e ? Hs : nullptr, s);
         }));
       } else {
         // this rank's share of dH_c in fp32, summed over ranks, then bf16
-        chk(L(KID_DH_F32, 0, (double)Tc * d * (4.0 * P.n_split + 4.0), [&] {
-          launch_dh_reduce_f32(b.dHp, P.n_split, (int64_t)Tc * d, dhf, s);
+        chk(L(KID_DH_F32, 0, (double)Tc * d * (4.0 * P.n_split + 4.0 + (store_e ? 4.0 : 0.0)),
+              [&] {
+          launch_dh_reduce_f32(b.dHp, P.n_split, (int64_t)Tc * d, dhf, d,
+                               store_e ? b.cst : nullptr, reinterpret_cast<const uint16_t*>(Hc),
+                               store_e ? Hs : nullptr, s);
         }));
         reduce();
         chk(L(KID_TO_BF16, 0, (double)Tc * d * 6.0, [&] {

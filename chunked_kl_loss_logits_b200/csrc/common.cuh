@@ -15,6 +15,11 @@ namespace ckl {
 // Device status bits (folded into ckl_status by the host).
 enum : unsigned { ST_INDEX_RANGE = 1u, ST_TIMEOUT = 2u, ST_INTERNAL = 4u };
 
+// Stored-exp backward: the largest distance (log2 units) a vocabulary tile's maximum
+// logit may lie above the row's reference logit before that tile stores its exps
+// relative to its own maximum instead (so every stored exp stays below 2^kRefGap).
+constexpr float kRefGap = 32.f;
+
 // A wait gives up after this many SM cycles (about two seconds at 1.9 GHz); every
 // pipeline step of a correct run completes within microseconds.
 constexpr long long kWaitCycles = 4000000000LL;

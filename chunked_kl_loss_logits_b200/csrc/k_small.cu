@@ -41,6 +41,16 @@ __device__ __forceinline__ float dot16(const uint4& a, const uint4& b, const flo
 constexpr int kGatherWarps = 4;
 constexpr int kTeacherWarps = 8;
 
+__host__ __device__ __forceinline__ int pow2_at_least(int k) {
+  int p = 1;
+  while (p < k) p <<= 1;
+  return p;
+}
+// Shared memory of one teacher warp: ids and logits (k_bytes each), then the sort keys.
+__host__ __device__ __forceinline__ size_t teacher_warp_bytes(int K, int k_bytes) {
+  return 2 * (size_t)k_bytes + 8 * (size_t)pow2_at_least(K);
+}
+
 // One warp per token of the chunk (bf16 path):
 //  1. stage the token's K ids and logits (16-byte loads when K % 4 == 0)
 //  2. p = softmax(logits); M = sum p; P_k = total p of slot k's id (repeats add)
@@ -52,15 +62,19 @@ constexpr int kTeacherWarps = 8;
 // the vocabulary is split over ranks), so ids outside the slice match no column.
 __global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ logit, int64_t t0, int Tc,
-    int V_all, int v0, int K, int k_bytes, float4* __restrict__ tok, float* __restrict__ Pk_out,
-    int32_t* __restrict__ sid_out, float* __restrict__ sp_out, unsigned* status) {
+    int V_all, int v0, int V_loc, int K, int k_bytes, float4* __restrict__ tok,
+    float* __restrict__ Pk_out, int32_t* __restrict__ sid_out, float* __restrict__ sp_out,
+    unsigned* status, const uint16_t* __restrict__ Hc, const uint16_t* __restrict__ W, int d,
+    int* __restrict__ rep) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * kTeacherWarps + warp;
+  if (rep && blockIdx.x == 0 && threadIdx.x == 0) rep[0] = 0;  // this chunk's repair list
   if (i >= Tc) return;
   const int64_t t = t0 + i;
-  int* sId = reinterpret_cast<int*>(smem + (size_t)warp * 2 * k_bytes);
-  float* sP = reinterpret_cast<float*>(smem + (size_t)warp * 2 * k_bytes + k_bytes);
+  int* sId = reinterpret_cast<int*>(smem + (size_t)warp * teacher_warp_bytes(K, k_bytes));
+  float* sP = reinterpret_cast<float*>(smem + (size_t)warp * teacher_warp_bytes(K, k_bytes) +
+                                       k_bytes);
 
   const int32_t* idr = idx + t * K;
   const float* lgr = logit + t * K;
@@ -76,6 +90,41 @@ __global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
     }
   }
   __syncwarp();
+  // Reference logit of the stored-exp backward: the student's logit (log2 units) at
+  // the slot with the largest teacher logit among the ids of this caller's rows,
+  // -inf when there is none. A logit at an actual id is at most the row's maximum,
+  // so exp(z - reference) can only overflow when the maximum lies far above it,
+  // which the forward epilogue checks tile by tile.
+  float r2 = 0.f;
+  if (Hc) {
+    float best = -INFINITY;
+    int bslot = K;
+    for (int k = lane; k < K; k += 32) {
+      const int id = sId[k] - v0;
+      if (id >= 0 && id < V_loc && sP[k] > best) { best = sP[k]; bslot = k; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int os = __shfl_xor_sync(0xffffffffu, bslot, o);
+      if (ob > best || (ob == best && os < bslot)) { best = ob; bslot = os; }
+    }
+    if (bslot < K) {
+      const uint4* hr = reinterpret_cast<const uint4*>(Hc + (int64_t)i * d);
+      const uint4* wr = reinterpret_cast<const uint4*>(W + (int64_t)(sId[bslot] - v0) * d);
+      float z = 0.f;
+      for (int c = lane; c < (d >> 3); c += 32) {
+        const uint4 a = __ldg(hr + c), b = __ldg(wr + c);
+        z = fmaf(lo_bf16(a.x), lo_bf16(b.x), z); z = fmaf(hi_bf16(a.x), hi_bf16(b.x), z);
+        z = fmaf(lo_bf16(a.y), lo_bf16(b.y), z); z = fmaf(hi_bf16(a.y), hi_bf16(b.y), z);
+        z = fmaf(lo_bf16(a.z), lo_bf16(b.z), z); z = fmaf(hi_bf16(a.z), hi_bf16(b.z), z);
+        z = fmaf(lo_bf16(a.w), lo_bf16(b.w), z); z = fmaf(hi_bf16(a.w), hi_bf16(b.w), z);
+      }
+      r2 = warp_sum(z) * 1.4426950408889634f;
+    } else {
+      r2 = -INFINITY;
+    }
+  }
   float mx = -INFINITY;
   for (int k = lane; k < K; k += 32) mx = fmaxf(mx, sP[k]);
   mx = warp_max(mx);
@@ -89,33 +138,59 @@ __global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
     const int id = sId[k];
     if (id < 0 || id >= V_all) atomicOr(status, (unsigned)ST_INDEX_RANGE);
   }
+  // Sort the (id, slot) pairs by id, ties in slot order: a bitonic network over the
+  // next power of two >= K of 64-bit keys (signed id, sign bit flipped, above the
+  // slot; padding keys sort last). The sorted order is what the forward epilogue
+  // walks, and equal ids become runs whose first slot carries their pooled P.
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(
+      smem + (size_t)warp * teacher_warp_bytes(K, k_bytes) + 2 * k_bytes);
+  const int Pk2 = pow2_at_least(K);
+  for (int k = lane; k < Pk2; k += 32)
+    key[k] = k < K ? ((unsigned long long)((uint32_t)sId[k] ^ 0x80000000u) << 32) | (uint32_t)k
+                   : ~0ull;
+  __syncwarp();
+  for (int size = 2; size <= Pk2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int j = lane; j < Pk2; j += 32) {
+        const int partner = j ^ stride;
+        if (partner > j) {
+          const unsigned long long a = key[j], b = key[partner];
+          if ((a > b) == ((j & size) == 0)) {
+            key[j] = b;
+            key[partner] = a;
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+  // Per sorted position: the run of equal ids around it (one entry unless an id
+  // repeats), its pooled probability P (summed in slot order), the sorted outputs,
+  // and P per slot for the entropy term (kept in sId's place, no longer needed).
+  float* sMP = reinterpret_cast<float*>(sId);
+  for (int j = lane; j < K; j += 32) {
+    const uint32_t hi = (uint32_t)(key[j] >> 32);
+    const int slot = (int)(uint32_t)key[j];
+    int st = j;
+    while (st > 0 && (uint32_t)(key[st - 1] >> 32) == hi) --st;
+    float P = 0.f;
+    for (int m = st; m < K && (uint32_t)(key[m] >> 32) == hi; ++m) P += sP[(uint32_t)key[m]];
+    const float p = sP[slot];
+    sMP[slot] = P;
+    Pk_out[(int64_t)i * K + slot] = st == j ? P : 0.f;
+    sid_out[(int64_t)i * K + j] = (int)(hi ^ 0x80000000u) - v0;
+    sp_out[(int64_t)i * K + j] = p;
+  }
   __syncwarp();
   float ent = 0.f, Msum = 0.f;
   for (int k = lane; k < K; k += 32) {
-    const int id = sId[k];
     const float p = sP[k];
-    float P = 0.f;
-    int rank = 0;
-    bool first = true;
-    for (int j = 0; j < K; ++j) {
-      const int o = sId[j];
-      if (o == id) {
-        P += sP[j];
-        first = first && (j >= k);
-        rank += j < k;
-      } else {
-        rank += o < id;
-      }
-    }
-    if (p > 0.f) ent += p * logf(P);
+    if (p > 0.f) ent += p * logf(sMP[k]);
     Msum += p;
-    Pk_out[(int64_t)i * K + k] = first ? P : 0.f;
-    sid_out[(int64_t)i * K + rank] = id - v0;
-    sp_out[(int64_t)i * K + rank] = p;
   }
   ent = warp_sum(ent);
   Msum = warp_sum(Msum);
-  if (lane == 0) tok[i] = make_float4(ent, 0.f, Msum, 0.f);
+  if (lane == 0) tok[i] = make_float4(ent, 0.f, Msum, r2);
 }
 
 // One warp per token of the chunk.
@@ -253,18 +328,32 @@ constexpr int kCombTok = 32, kCombSplit = 32;
 
 // From a token's merged (max, sum) in log2 units and its cross term: lse,
 // l_t = ent - cross + M lse and the gradient multipliers.
+// With `rep` (stored-exp backward): the row's reference R for the stored exp(z - R),
+// in log2 units, is the teacher kernel's reference r2 unless some tile of this
+// caller's rows has its maximum more than kRefGap above r2 (local_M2, the largest
+// tile maximum, tells); such a tile stored exp(z - its own maximum), so the row
+// joins the repair list and R becomes local_M2. cst.w = R.
 __device__ __forceinline__ void finish_token(int64_t t0, int i, float M2, float S, float cross,
                                              const uint8_t* __restrict__ mask,
                                              const float4* __restrict__ tok,
                                              const Misc* __restrict__ misc, float4* __restrict__ cst,
                                              float* __restrict__ lse_all,
-                                             float* __restrict__ ell_all) {
+                                             float* __restrict__ ell_all, float local_M2,
+                                             int* __restrict__ rep) {
   const float lse = (M2 + log2f(S)) * kLn2;
   const float4 t4 = tok[i];
   const float ell = t4.x - cross + t4.z * lse;
   const int64_t t = t0 + i;
   const float sc = (mask == nullptr || mask[t] != 0) ? misc->invN : 0.f;
-  cst[i] = make_float4(lse, sc * t4.z, sc, 0.f);
+  float R = 0.f;
+  if (rep) {
+    R = t4.w;
+    if (local_M2 > t4.w + kRefGap) {
+      R = local_M2;
+      rep[1 + atomicAdd(rep, 1)] = i;
+    }
+  }
+  cst[i] = make_float4(lse, sc * t4.z, sc, R);
   lse_all[t] = lse;
   ell_all[t] = ell;
 }
@@ -280,7 +369,7 @@ __global__ void __launch_bounds__(kCombTok * kCombSplit) combine_kernel(
     const float2* __restrict__ part, const float* __restrict__ xpart,
     const float4* __restrict__ tok, const Misc* __restrict__ misc,
     float4* __restrict__ cst, float* __restrict__ lse_all, float* __restrict__ ell_all,
-    float4* __restrict__ stats) {
+    float4* __restrict__ stats, int* __restrict__ rep) {
   __shared__ float sm[kCombSplit][kCombTok], ss[kCombSplit][kCombTok], sx[kCombSplit][kCombTok];
   const int tk = threadIdx.x % kCombTok, sp = threadIdx.x / kCombTok;
   const int i = blockIdx.x * kCombTok + tk;
@@ -317,16 +406,18 @@ __global__ void __launch_bounds__(kCombTok * kCombSplit) combine_kernel(
     stats[i] = make_float4(M2, S, cross, 0.f);
     return;
   }
-  finish_token(t0, i, M2, S, cross, mask, tok, misc, cst, lse_all, ell_all);
+  finish_token(t0, i, M2, S, cross, mask, tok, misc, cst, lse_all, ell_all, M2, rep);
 }
 
 // Vocabulary split over ranks: merge every rank's (max, sum, cross) of a token,
 // in rank order (stats_all is rank-major, world x Tc), so that every rank
 // computes the same lse and l_t bit for bit. One thread per token.
-__global__ void vp_merge_kernel(int64_t t0, int Tc, int world, const float4* __restrict__ stats_all,
+__global__ void vp_merge_kernel(int64_t t0, int Tc, int world, int rank,
+                                const float4* __restrict__ stats_all,
                                 const uint8_t* __restrict__ mask, const float4* __restrict__ tok,
                                 const Misc* __restrict__ misc, float4* __restrict__ cst,
-                                float* __restrict__ lse_all, float* __restrict__ ell_all) {
+                                float* __restrict__ lse_all, float* __restrict__ ell_all,
+                                int* __restrict__ rep) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= Tc) return;
   float M2 = -INFINITY;
@@ -337,40 +428,45 @@ __global__ void vp_merge_kernel(int64_t t0, int Tc, int world, const float4* __r
     if (q.x > -INFINITY) S += q.y * ex2_approx(q.x - M2);
     X += q.z;
   }
-  finish_token(t0, i, M2, S, X, mask, tok, misc, cst, lse_all, ell_all);
+  // the reference and the stored exps are this rank's own: its rows' largest tile max
+  finish_token(t0, i, M2, S, X, mask, tok, misc, cst, lse_all, ell_all,
+               stats_all[(int64_t)rank * Tc + i].x, rep);
 }
 
-// Stored-exp forward: the (blocked, bf16) gradient buffer holds
-// e = exp2(z log2e - m2_tile); turn it into G = gmul exp(z - lse)
-// = e * gmul * exp2(m2_tile - lse log2e) in place. One CUDA block per 64 x 64
-// element block of G (8 KB contiguous); each thread loads two 16-byte groups
-// (rows r and r + 32) before scaling either.
-__global__ void __launch_bounds__(256) scale_e_kernel(uint16_t* __restrict__ G, int n_vb, int Tc,
-                                                      int V, const float2* __restrict__ part,
-                                                      const float4* __restrict__ cst) {
-  const int vb = blockIdx.x, tb = blockIdx.y;
-  uint16_t* blk = G + ((int64_t)tb * n_vb + vb) * 4096;
-  const int c = (threadIdx.x & 7) * 8;            // first of the group's 8 columns
-  const int v = vb * 64 + c;
-  const int r0 = threadIdx.x >> 3;                // rows r0 and r0 + 32 of the block
-  const int t[2] = {tb * 64 + r0, tb * 64 + r0 + 32};
-  uint4 x[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-  if (v >= V) return;
-#pragma unroll
-  for (int u = 0; u < 2; ++u)
-    if (t[u] < Tc) x[u] = *reinterpret_cast<const uint4*>(blk + (r0 + 32 * u) * 64 + c);
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    if (t[u] >= Tc) continue;
-    const float4 cc = cst[t[u]];
-    const float f = cc.y * ex2_approx(part[(int64_t)(v >> 8) * Tc + t[u]].x -
-                                      cc.x * 1.4426950408889634f);
-    uint4 y = x[u];
+// Stored-exp backward, rows on the repair list: the forward epilogue stored
+// exp2(z log2e - ref_j) in each vocabulary tile j, with ref_j the tile's maximum m2_j
+// when m2_j > r2 + kRefGap and the row's reference r2 otherwise; the row's common
+// reference is now R = cst.w (the largest tile maximum), so every stored value is
+// multiplied by exp2(ref_j - R) <= 1, in place. Rows not on the list need nothing.
+// A fixed grid strides over (listed rows) x (64-wide vocabulary blocks) x 8 groups
+// of 8 elements; with an empty list every thread reads the count and returns.
+__global__ void __launch_bounds__(256) repair_kernel(uint16_t* __restrict__ G, int n_vb, int Tc,
+                                                     int V, const float2* __restrict__ part,
+                                                     const float4* __restrict__ cst,
+                                                     const float4* __restrict__ tok,
+                                                     const int* __restrict__ rep) {
+  const int n = rep[0];
+  const int64_t per_row = (int64_t)n_vb * 8;
+  const int64_t total = (int64_t)n * per_row;
+  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < total;
+       it += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(it / per_row);
+    const int rem = (int)(it - (int64_t)r * per_row);
+    const int vb = rem >> 3, c = (rem & 7) * 8;
+    const int v = vb * 64 + c;
+    if (v >= V) continue;
+    const int t = rep[1 + r];
+    const float R = cst[t].w, r2 = tok[t].w;
+    const float m2 = part[(int64_t)(v >> 8) * Tc + t].x;
+    const float f = ex2_approx((m2 > r2 + kRefGap ? m2 : r2) - R);
+    uint4* q = reinterpret_cast<uint4*>(G + (((int64_t)(t >> 6) * n_vb + vb) << 12) +
+                                        ((t & 63) << 6) + c);
+    uint4 y = *q;
     y.x = pack_bf16x2(lo_bf16(y.x) * f, hi_bf16(y.x) * f);
     y.y = pack_bf16x2(lo_bf16(y.y) * f, hi_bf16(y.y) * f);
     y.z = pack_bf16x2(lo_bf16(y.z) * f, hi_bf16(y.z) * f);
     y.w = pack_bf16x2(lo_bf16(y.w) * f, hi_bf16(y.w) * f);
-    *reinterpret_cast<uint4*>(blk + (r0 + 32 * u) * 64 + c) = y;
+    *q = y;
   }
 }
 
@@ -391,15 +487,17 @@ __device__ __forceinline__ float load_g(const uint16_t* G, int64_t off) {
   return bf16_to_f32(G[off]);
 }
 
-// One thread per (token, slot) that holds the first occurrence of an id (P_k > 0):
-// overwrite: G[i][id] = gmul exp(z_k - lse) - s P_k;  else: G[i][id] -= s P_k.
+// One thread per (token, slot) that holds the first occurrence of an id (P_k > 0).
+// G holds gmul exp(z - lse): G[i][id] -= s P_k. With `row_ref` G holds the stored
+// exp(z - R) instead, the gradient being c exp(z - R) with c = gmul exp(R - lse):
+// G[i][id] -= (P_k / M) exp(lse - R), so that c times it is the gradient there.
 // Ids are taken relative to v0 (the slice's first row); ids outside [0, V) of
 // the slice belong to another rank and are skipped.
 template <typename Tg>
 __global__ void fixup_kernel(const int32_t* __restrict__ idx, int64_t t0, int Tc, int K, int V,
                              int v0, int64_t ldG, const float4* __restrict__ cst,
-                             const float* __restrict__ zk, const float* __restrict__ Pk, Tg* G,
-                             int overwrite) {
+                             const float4* __restrict__ tok, const float* __restrict__ Pk, Tg* G,
+                             int row_ref) {
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= (int64_t)Tc * K) return;
   const float P = Pk[e];
@@ -409,22 +507,51 @@ __global__ void fixup_kernel(const int32_t* __restrict__ idx, int64_t t0, int Tc
   if (id < 0 || id >= V) return;
   const float4 c = cst[i];
   const int64_t off = g_off(G, i, id, ldG);
-  const float g = overwrite ? c.y * expf(zk[e] - c.x) - c.z * P : load_g(G, off) - c.z * P;
-  store_g(G, off, g);
+  const float sub = row_ref ? (P / tok[i].z) * ex2_approx(c.x * 1.4426950408889634f - c.w)
+                            : c.z * P;
+  store_g(G, off, load_g(G, off) - sub);
 }
 
 // Sum of the split-K partials in fp32 (vocabulary split over ranks: the ranks'
 // sums are added by the exchange before the conversion to bf16).
+// Stored-exp backward: the row factor c_t = gmul exp2(R - lse log2e) that turns the
+// stored exp(z - R) into the gradient (0 for masked tokens); 1 when G is the gradient.
+__device__ __forceinline__ float row_factor(const float4* __restrict__ cst, int64_t t) {
+  if (!cst) return 1.f;
+  const float4 q = cst[t];
+  return q.y * ex2_approx(q.w - q.x * 1.4426950408889634f);
+}
+
+// Hs[t] = bf16(c_t H[t]) for 8 elements at e8: DW then contracts the stored exps
+// with the scaled hidden states (dW = sum_t exp(z_t - R_t)^T (c_t H_t)).
+__device__ __forceinline__ void scale_h8(const uint16_t* __restrict__ Hc, uint16_t* __restrict__ Hs,
+                                         int64_t e8, float c) {
+  const uint4 x = *reinterpret_cast<const uint4*>(Hc + e8);
+  uint4 y;
+  y.x = pack_bf16x2(lo_bf16(x.x) * c, hi_bf16(x.x) * c);
+  y.y = pack_bf16x2(lo_bf16(x.y) * c, hi_bf16(x.y) * c);
+  y.z = pack_bf16x2(lo_bf16(x.z) * c, hi_bf16(x.z) * c);
+  y.w = pack_bf16x2(lo_bf16(x.w) * c, hi_bf16(x.w) * c);
+  *reinterpret_cast<uint4*>(Hs + e8) = y;
+}
+
 __global__ void dh_reduce_f32_kernel(const float* __restrict__ dHp, int n_split, int64_t n_elem,
-                                     float* __restrict__ out) {
-  const int64_t e4 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
-  if (e4 >= n_elem) return;
-  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+                                     float* __restrict__ out, int d, const float4* __restrict__ cst,
+                                     const uint16_t* __restrict__ Hc, uint16_t* __restrict__ Hs) {
+  const int64_t e8 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (e8 >= n_elem) return;
+  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (int s = 0; s < n_split; ++s) {
-    const float4 x = *reinterpret_cast<const float4*>(dHp + s * n_elem + e4);
-    a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+    const float4* p = reinterpret_cast<const float4*>(dHp + s * n_elem + e8);
+    const float4 x = p[0], y = p[1];
+    a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
+    a[4] += y.x; a[5] += y.y; a[6] += y.z; a[7] += y.w;
   }
-  *reinterpret_cast<float4*>(out + e4) = a;
+  const float c = row_factor(cst, e8 / d);
+  float4* o = reinterpret_cast<float4*>(out + e8);
+  o[0] = make_float4(a[0] * c, a[1] * c, a[2] * c, a[3] * c);
+  o[1] = make_float4(a[4] * c, a[5] * c, a[6] * c, a[7] * c);
+  if (Hs) scale_h8(Hc, Hs, e8, c);
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ in, int64_t n_elem,
@@ -439,7 +566,9 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ in, int64_t n_elem,
 }
 
 __global__ void dh_reduce_bf16_kernel(const float* __restrict__ dHp, int n_split, int64_t n_elem,
-                                      uint16_t* __restrict__ dH) {
+                                      uint16_t* __restrict__ dH, int d,
+                                      const float4* __restrict__ cst,
+                                      const uint16_t* __restrict__ Hc, uint16_t* __restrict__ Hs) {
   const int64_t e8 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (e8 >= n_elem) return;
   float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -449,6 +578,12 @@ __global__ void dh_reduce_bf16_kernel(const float* __restrict__ dHp, int n_split
     a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
     a[4] += y.x; a[5] += y.y; a[6] += y.z; a[7] += y.w;
   }
+  const float c = row_factor(cst, e8 / d);
+  if (cst) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] *= c;
+  }
+  if (Hs) scale_h8(Hc, Hs, e8, c);
   uint4 o;
   o.x = pack_bf16x2(a[0], a[1]);
   o.y = pack_bf16x2(a[2], a[3]);
@@ -654,13 +789,15 @@ void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t 
 }
 
 void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V_all, int v0,
-                    int K, const ChunkBufs& b, unsigned* status, cudaStream_t s) {
+                    int V_loc, int K, const ChunkBufs& b, unsigned* status, const uint16_t* Hc,
+                    const uint16_t* W, int d, cudaStream_t s) {
   const int k_bytes = (K * 4 + 15) & ~15;
-  const size_t smem = (size_t)kTeacherWarps * 2 * k_bytes;
+  const size_t smem = (size_t)kTeacherWarps * teacher_warp_bytes(K, k_bytes);
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(teacher_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   teacher_kernel<<<blocks_for(Tc, kTeacherWarps), kTeacherWarps * 32, smem, s>>>(
-      idx, logit, t0, Tc, V_all, v0, K, k_bytes, b.tok, b.Pk, b.sid, b.sp, status);
+      idx, logit, t0, Tc, V_all, v0, V_loc, K, k_bytes, b.tok, b.Pk, b.sid, b.sp, status, Hc, W,
+      d, Hc ? b.rep : nullptr);
 }
 
 template <typename Tin>
@@ -682,42 +819,46 @@ template void launch_gather<float>(const float*, const float*, const int32_t*, c
                                    cudaStream_t);
 
 void launch_combine(int64_t t0, int Tc, int n_vt, const uint8_t* mask, const ChunkBufs& b,
-                    float* lse_all, float* ell_all, float4* stats, cudaStream_t s) {
+                    float* lse_all, float* ell_all, float4* stats, bool row_ref, cudaStream_t s) {
   combine_kernel<<<blocks_for(Tc, kCombTok), kCombTok * kCombSplit, 0, s>>>(
-      t0, Tc, n_vt, mask, b.part, b.xpart, b.tok, b.misc, b.cst, lse_all, ell_all, stats);
+      t0, Tc, n_vt, mask, b.part, b.xpart, b.tok, b.misc, b.cst, lse_all, ell_all, stats,
+      row_ref ? b.rep : nullptr);
 }
 
-void launch_vp_merge(int64_t t0, int Tc, int world, const float4* stats_all, const uint8_t* mask,
-                     const ChunkBufs& b, float* lse_all, float* ell_all, cudaStream_t s) {
-  vp_merge_kernel<<<blocks_for(Tc, 128), 128, 0, s>>>(t0, Tc, world, stats_all, mask, b.tok,
-                                                      b.misc, b.cst, lse_all, ell_all);
+void launch_vp_merge(int64_t t0, int Tc, int world, int rank, const float4* stats_all,
+                     const uint8_t* mask, const ChunkBufs& b, float* lse_all, float* ell_all,
+                     bool row_ref, cudaStream_t s) {
+  vp_merge_kernel<<<blocks_for(Tc, 128), 128, 0, s>>>(t0, Tc, world, rank, stats_all, mask, b.tok,
+                                                      b.misc, b.cst, lse_all, ell_all,
+                                                      row_ref ? b.rep : nullptr);
 }
 
-void launch_scale_e(uint16_t* G, int Tc, int V, const ChunkBufs& b, cudaStream_t s) {
+void launch_repair(uint16_t* G, int Tc, int V, const ChunkBufs& b, int num_sms, cudaStream_t s) {
   const int n_vb = (V + 63) / 64;
-  const dim3 grid((unsigned)n_vb, (unsigned)((Tc + 63) / 64));
-  scale_e_kernel<<<grid, 256, 0, s>>>(G, n_vb, Tc, V, b.part, b.cst);
+  repair_kernel<<<2 * num_sms, 256, 0, s>>>(G, n_vb, Tc, V, b.part, b.cst, b.tok, b.rep);
 }
 
 template <typename Tg>
 void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int v0, int64_t ldG,
-                  const ChunkBufs& b, bool overwrite, cudaStream_t s) {
+                  const ChunkBufs& b, bool row_ref, cudaStream_t s) {
   fixup_kernel<Tg><<<blocks_for((int64_t)Tc * K, 256), 256, 0, s>>>(
-      idx, t0, Tc, K, V, v0, ldG, b.cst, b.zk, b.Pk, static_cast<Tg*>(b.G), overwrite ? 1 : 0);
+      idx, t0, Tc, K, V, v0, ldG, b.cst, b.tok, b.Pk, static_cast<Tg*>(b.G), row_ref ? 1 : 0);
 }
 template void launch_fixup<float>(const int32_t*, int64_t, int, int, int, int, int64_t,
                                   const ChunkBufs&, bool, cudaStream_t);
 template void launch_fixup<uint16_t>(const int32_t*, int64_t, int, int, int, int, int64_t,
                                      const ChunkBufs&, bool, cudaStream_t);
 
-void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
-                           cudaStream_t s) {
-  dh_reduce_bf16_kernel<<<blocks_for(n_elem / 8, 256), 256, 0, s>>>(dHp, n_split, n_elem, dH);
+void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH, int d,
+                           const float4* cst, const uint16_t* Hc, uint16_t* Hs, cudaStream_t s) {
+  dh_reduce_bf16_kernel<<<blocks_for(n_elem / 8, 256), 256, 0, s>>>(dHp, n_split, n_elem, dH, d,
+                                                                    cst, Hc, Hs);
 }
 
-void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out,
-                          cudaStream_t s) {
-  dh_reduce_f32_kernel<<<blocks_for(n_elem / 4, 256), 256, 0, s>>>(dHp, n_split, n_elem, out);
+void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out, int d,
+                          const float4* cst, const uint16_t* Hc, uint16_t* Hs, cudaStream_t s) {
+  dh_reduce_f32_kernel<<<blocks_for(n_elem / 8, 256), 256, 0, s>>>(dHp, n_split, n_elem, out, d,
+                                                                   cst, Hc, Hs);
 }
 
 void launch_f32_to_bf16(const float* in, int64_t n_elem, uint16_t* out, cudaStream_t s) {

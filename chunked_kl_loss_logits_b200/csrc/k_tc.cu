@@ -8,8 +8,8 @@
 //   LSE : z = H_c W^T tile by tile; the epilogue keeps each row's (max, sum of
 //         exp) over the tile's vocabulary columns, and sum_k p_k z_k over the
 //         row's cached teacher ids that fall in the tile. With `store_e` it also writes
-//         e = exp(z - tile max) in bf16 to the chunk's gradient buffer, so the
-//         backward pass can rescale it instead of forming z again.
+//         exp(z - r) in bf16 to the chunk's gradient buffer (r the row's reference
+//         logit), so the backward pass can scale rows instead of forming z again.
 //   GRAD: z formed again; the epilogue writes G = gmul * exp(z - lse) in bf16.
 //   DH  : dH_c = G W, the vocabulary split in n_split ranges (fp32 partials,
 //         reduced in a fixed order afterwards).
@@ -393,7 +393,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               s += (cb + j < p.V) ? ex2_approx(fmaf(v[j], kLog2e, -m2)) : 0.f;
           }
         } else {
-          // e = exp2(z log2e - m2) in (0, 1], stored as bf16 64 columns at a time
+          // e = exp2(z log2e - m2) in (0, 1] enters the sum; the value stored (bf16, 64
+          // columns at a time) is e * exp2(m2 - ref) = exp2(z log2e - ref), with ref the
+          // row's reference unless this tile's maximum lies more than kRefGap above it
+          const float r2 = row_ok ? p.tok[grow].w : m2;
+          const float ref = m2 > r2 + kRefGap ? m2 : r2;
+          const float fs = ex2_approx(m2 - ref);
 #pragma unroll 1
           for (int cc = 0; cc < BN / 64; ++cc) {
             float a[32], b[32];
@@ -413,6 +418,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               s += b[j];
             }
             if (cb < p.V) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                a[j] *= fs;
+                b[j] *= fs;
+              }
               uint4 ch[8];
               pack_row_bf16(a, b, ch);
               stage_and_issue(ch, cb, row0, false);

@@ -24,7 +24,10 @@ struct TcLaunch {
   const float* sp;     // LSE: their teacher probabilities
   float* xpart;        // LSE: per-tile partial cross term, same layout as part
   int K;
-  int store_e;     // LSE: also store exp(z - tile max) in bf16 through map c
+  int store_e;     // LSE: also store exp(z - ref) in bf16 through map c, with ref the
+                   // row's reference tok[row].w (log2 units), or the tile's maximum when
+                   // that lies more than kRefGap above it
+  const float4* tok;  // LSE with store_e: per-row values, .w = the reference
   const float4* cst;  // GRAD
   uint16_t* G;        // GRAD
   int64_t ldG;        // GRAD

@@ -10,8 +10,10 @@
 namespace ckl {
 
 // Per-token values of the chunk being processed, in the workspace.
-//   tok[i] = (ent_i, cross_i, M_i, 0)   from the teacher gather
-//   cst[i] = (lse_i, gmul_i, s_i, 0)    from the combine: gmul = s * M, s = mask/N
+//   tok[i] = (ent_i, cross_i, M_i, r2_i)   from the teacher kernel; r2 = the reference
+//            logit of the stored-exp backward (log2 units; 0 when not used)
+//   cst[i] = (lse_i, gmul_i, s_i, R_i)     from the combine: gmul = s * M, s = mask/N,
+//            R = the row's reference of the stored exps (stored-exp backward only)
 struct Misc;
 struct ChunkBufs {
   float4* tok;
@@ -25,6 +27,7 @@ struct ChunkBufs {
   float* sp;     // bf16: Tc x K teacher probability of each sorted slot
   void* G;       // Tc x ldG scaled gradient of the logits (bf16 or f32)
   float* dHp;    // split-K partials of dH (bf16 path)
+  int* rep;      // stored-exp backward: [count, rows...] of the rows to repair this chunk
   struct Misc* misc;
 };
 
@@ -41,31 +44,42 @@ void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t 
 // bf16: teacher softmax, merged P, entropy term and each token's ids sorted with
 // their probabilities (the forward contraction picks the student logits there).
 // Ids are checked against V_all and written relative to v0 (vocabulary split
-// over ranks: this rank holds rows [v0, v0 + V) of W; otherwise v0 = 0, V_all = V).
+// over ranks: this rank holds rows [v0, v0 + V_loc) of W; otherwise v0 = 0,
+// V_all = V_loc). With Hc (the chunk's hidden states; W and d then too): also the
+// reference logit r2 of the stored-exp backward into tok.w, and the chunk's
+// repair list is emptied.
 void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V_all, int v0,
-                    int K, const ChunkBufs& b, unsigned* status, cudaStream_t s);
+                    int V_loc, int K, const ChunkBufs& b, unsigned* status, const uint16_t* Hc,
+                    const uint16_t* W, int d, cudaStream_t s);
 // fp32: as launch_teacher, plus the student logits at the ids by dot products.
 template <typename Tin>
 void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* logit, int64_t t0,
                    int Tc, int d, int V, int K, const ChunkBufs& b, unsigned* status,
                    cudaStream_t s);
 // stats != nullptr: write this rank's per-token (max2, sum, cross, 0) and stop.
+// row_ref (stored-exp backward): also each row's reference R into cst.w, rows whose
+// tiles outgrew the teacher kernel's reference joining the repair list.
 void launch_combine(int64_t t0, int Tc, int n_vt, const uint8_t* mask, const ChunkBufs& b,
-                    float* lse_all, float* ell_all, float4* stats, cudaStream_t s);
-// Merge world x Tc gathered stats (rank-major) into lse, l_t and the multipliers.
-void launch_vp_merge(int64_t t0, int Tc, int world, const float4* stats_all, const uint8_t* mask,
-                     const ChunkBufs& b, float* lse_all, float* ell_all, cudaStream_t s);
-// G at the cached ids. overwrite: G = gmul exp(z_k - lse) - s P_k (the gradient
-// contraction wrote gmul exp(z - lse) there); otherwise G -= s P_k in place.
+                    float* lse_all, float* ell_all, float4* stats, bool row_ref, cudaStream_t s);
+// Merge world x Tc gathered stats (rank-major) into lse, l_t and the multipliers
+// (and, with row_ref, this rank's row references and repair list).
+void launch_vp_merge(int64_t t0, int Tc, int world, int rank, const float4* stats_all,
+                     const uint8_t* mask, const ChunkBufs& b, float* lse_all, float* ell_all,
+                     bool row_ref, cudaStream_t s);
+// G at the cached ids, in place: G -= s P_k where G is gmul exp(z - lse); with
+// row_ref (G holds the stored exp(z - R)) G -= (P_k / M) exp(lse - R).
 template <typename Tg>
 // ldG: fp32 row stride of G; bf16: the number of 64-wide vocabulary blocks (G blocked).
 void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int v0, int64_t ldG,
-                  const ChunkBufs& b, bool overwrite, cudaStream_t s);
-// Stored-exp forward: G[i][v] = e[i][v] * gmul_i * exp2(m2[tile(v)][i] - lse_i log2 e), in place
-// (G blocked, bf16).
-void launch_scale_e(uint16_t* G, int Tc, int V, const ChunkBufs& b, cudaStream_t s);
-void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH,
-                           cudaStream_t s);
+                  const ChunkBufs& b, bool row_ref, cudaStream_t s);
+// Stored-exp backward: rescale the rows on the chunk's repair list to their common
+// reference R, in place (G blocked, bf16); nothing to do for an empty list.
+void launch_repair(uint16_t* G, int Tc, int V, const ChunkBufs& b, int num_sms, cudaStream_t s);
+// Sum of the n_split partials of dH_c -> bf16 dH. With cst (stored-exp backward)
+// each row is multiplied by c_t = gmul exp(R - lse), and Hs = bf16(c_t Hc) is written
+// for the dW contraction (Hs may be NULL).
+void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH, int d,
+                           const float4* cst, const uint16_t* Hc, uint16_t* Hs, cudaStream_t s);
 // One thread waits on a barrier nothing arrives at until the wait bound fires.
 void launch_wait_selftest(unsigned* status, long long* cycles, cudaStream_t s);
 // Top-K cache with the vocabulary split over ranks: pack this rank's K best as
@@ -74,9 +88,10 @@ void launch_topk_pack(const int32_t* idx, const float* lg, int64_t n, int v0, fl
                       cudaStream_t s);
 void launch_topk_regroup(const float2* gathered, int world, int rows, int K, float2* cand, int* cnt,
                          cudaStream_t s);
-// n_elem % 4 == 0
-void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out,
-                          cudaStream_t s);
+// As launch_dh_reduce_bf16 with an fp32 result (the vocabulary-parallel all-reduce's
+// buffer). n_elem % 8 == 0.
+void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out, int d,
+                          const float4* cst, const uint16_t* Hc, uint16_t* Hs, cudaStream_t s);
 void launch_f32_to_bf16(const float* in, int64_t n_elem, uint16_t* out, cudaStream_t s);
 // Teacher top-K cache: per row, the threshold = the K-th best of the n_vt tile
 // bests (logit descending, id ascending), or "take everything" when n_vt <= K.

@@ -86,7 +86,11 @@ def test_vocab_parallel_headline_shape():
     h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=2048)
     l1, dH1, dW1 = h.fwd_bwd(H, W, idx, logit, mask, chunk=2048)
     assert rel(loss.item(), l1.item()) <= 1e-6
+    # the gradients of the two calls agree to within their own bf16 rounding: each
+    # rank keeps its exps against a reference logit of its own rows (the single-rank
+    # call against the teacher's best id), so the bf16 exps and the scaled hidden
+    # states dW contracts them with are rounded differently (2^-9 relative each)
     dW = torch.cat([o[2] for o in out])
-    assert ((dW - dW1.cpu()).norm() / dW1.cpu().norm()).item() <= 1e-3
-    assert ((dH.float() - dH1.cpu().float()).norm() / dH1.cpu().float().norm()).item() <= 1e-3
+    assert ((dW - dW1.cpu()).norm() / dW1.cpu().norm()).item() <= 5e-3
+    assert ((dH.float() - dH1.cpu().float()).norm() / dH1.cpu().float().norm()).item() <= 5e-3
     h.close()
