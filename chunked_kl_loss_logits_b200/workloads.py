@@ -73,6 +73,11 @@ WORKLOADS = {
     # a 32000-word vocabulary, so W (184 MB) still exceeds L2 while the whole
     # footprint stays under 1 GB for multi-pass counter captures.
     "prof_2k": Workload("prof_2k", 2048, 2880, 32000, 100, 2048, "bf16", 3.0, "zipf", seed=1099),
+    # Two chunks of the same shapes: the second dW contraction adds into the dW the
+    # first one stored, as every chunk after the first does at full size (dW, 368 MB
+    # fp32, still exceeds L2).
+    "prof_2x2k": Workload("prof_2x2k", 4096, 2880, 32000, 100, 2048, "bf16", 3.0, "zipf",
+                          seed=1098),
 }
 
 _STREAMS = ("perm", "ids", "logits", "H", "W", "mask")
