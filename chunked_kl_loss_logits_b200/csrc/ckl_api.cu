@@ -115,10 +115,11 @@ struct WsPlan {
   size_t off_stats = 0, off_stats_all = 0, off_dhf = 0;
 };
 
-// dH tiles are 256 x 256 outputs computed by CTA pairs; split the vocabulary
+// dH tiles are 256 x tc_bn(DH) outputs computed by CTA pairs; split the vocabulary
 // (the contraction) so that the tile count fills the pairs evenly.
 int pick_dh_split(int64_t Tc, int64_t d, int64_t V, int num_sms) {
-  const int64_t tiles = ((Tc + 255) / 256) * ((d + 255) / 256);
+  const int tw = tc_bn(TcKind::DH);
+  const int64_t tiles = ((Tc + 255) / 256) * ((d + tw - 1) / tw);
   const int64_t n_kb = (V + 63) / 64;
   const int units = std::max(1, num_sms / 2);
   int best = 1;

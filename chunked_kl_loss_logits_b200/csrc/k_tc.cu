@@ -63,13 +63,20 @@ constexpr uint16_t kPairMask = 0x3;
 
 template <TcKind KIND>
 struct Cfg;
-// BN: output columns per pair tile (each CTA stages BN/2 rows or columns of B).
-template <> struct Cfg<TcKind::LSE>  { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
-template <> struct Cfg<TcKind::GRAD> { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
-template <> struct Cfg<TcKind::DH>   { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = true;  static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
-template <> struct Cfg<TcKind::DW>   { static constexpr int BN = 256; static constexpr bool A_MN = true,  B_MN = true;  static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
-template <> struct Cfg<TcKind::TKMAX>  { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
-template <> struct Cfg<TcKind::TKEMIT> { static constexpr int BN = 256; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
+// BN: output columns of one accumulator (each CTA stages BN/2 rows or columns of B).
+// NACC: accumulators per tile. DH runs two side by side (a 256 x 512 tile): every A
+// stage (G) feeds two MMAs, so a stage moves 48 KB per CTA for twice the work of a
+// 32 KB single-accumulator stage, and a vocabulary split has half as many tiles
+// (48 at the 32K workload, so the three splits' 144 tiles run as two waves on 74
+// pairs and far fewer tiles re-stream a split's G and W from DRAM). The two
+// accumulators fill all 512 TMEM columns, so that kind is single-buffered: its
+// tiles run ~1000 K-blocks, against an epilogue of a few microseconds.
+template <> struct Cfg<TcKind::LSE>  { static constexpr int BN = 256, NACC = 1; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::GRAD> { static constexpr int BN = 256, NACC = 1; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::DH>   { static constexpr int BN = 256, NACC = 2; static constexpr bool A_MN = false, B_MN = true;  static constexpr int STAGES = 4; static constexpr bool STAGED = false; };
+template <> struct Cfg<TcKind::DW>   { static constexpr int BN = 256, NACC = 1; static constexpr bool A_MN = true,  B_MN = true;  static constexpr int STAGES = 6; static constexpr bool STAGED = true; };
+template <> struct Cfg<TcKind::TKMAX>  { static constexpr int BN = 256, NACC = 1; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
+template <> struct Cfg<TcKind::TKEMIT> { static constexpr int BN = 256, NACC = 1; static constexpr bool A_MN = false, B_MN = false; static constexpr int STAGES = 7; static constexpr bool STAGED = false; };
 
 // The bf16 gradient buffer is blocked: 64 x 64 element blocks (64 vocabulary ids
 // fastest, then 64 tokens; 8 KB contiguous), seen by TMA as the 4-D tensor
@@ -87,9 +94,15 @@ struct Layout {
   static constexpr int BN = Cfg<KIND>::BN;
   static constexpr int BNH = BN / 2;
   static constexpr int STAGES = Cfg<KIND>::STAGES;
+  static constexpr int NACC = Cfg<KIND>::NACC;
+  static constexpr int TW = BN * NACC;                  // output columns of a tile
+  static constexpr int NBUF = NACC == 1 ? 2 : 1;        // accumulator buffers in TMEM
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BNH * BK * 2;
+  static constexpr int B_HALF_BYTES = BNH * BK * 2;     // one accumulator's B, this CTA's half
+  static constexpr int B_BYTES = NACC * B_HALF_BYTES;
   static_assert(!Cfg<KIND>::B_MN || BNH % 64 == 0, "MN-major B is staged in 64-column atoms");
+  static_assert(NACC * BN <= kTmemCols && (NBUF == 1 || NACC * BN <= kAccStride),
+                "accumulators fit in TMEM");
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   // two staging boxes per epilogue warp
@@ -160,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const __grid_constant__ CUtensorMap tmC, const TcLaunch p) {
   using L = Layout<KIND>;
   constexpr int STAGES = L::STAGES;
-  constexpr int BN = L::BN, BNH = L::BNH;
+  constexpr int BN = L::BN, BNH = L::BNH, TW = L::TW, NACC = L::NACC, NBUF = L::NBUF;
   constexpr bool A_MN = Cfg<KIND>::A_MN, B_MN = Cfg<KIND>::B_MN;
 
   extern __shared__ unsigned char smem_raw[];
@@ -180,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();  // 0: leader (issues MMAs), 1: peer
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   const int n_m = (p.M + 2 * BM - 1) / (2 * BM);
-  const int n_n = (p.N + BN - 1) / BN;
+  const int n_n = (p.N + TW - 1) / TW;
   const int n_split = (KIND == TcKind::DH) ? p.n_split : 1;
   const int kps = (p.n_kb + n_split - 1) / n_split;
   const int n_tiles = n_m * n_n * n_split;
@@ -220,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = pair; ok && tile < n_tiles; tile += n_pairs) {
         const TileCoord c = tile_coord(p, n_m, n_n, kps, tile);
         const int a_row0 = c.mt * 2 * BM + (int)rank * BM;  // this CTA's rows of A
-        const int b_row0 = c.nt * BN + (int)rank * BNH;     // this CTA's rows/columns of B
+        const int b_row0 = c.nt * TW + (int)rank * BNH;     // this CTA's rows/columns of B
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           unsigned char* sA = smem + stage * L::STAGE_BYTES;
@@ -241,12 +254,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int a = 0; a < BM / 64; ++a)
               tma_load_2d_pair(sA + a * kAtomBytes, &tmA, fbar, a_row0 + a * 64, kb * BK);
           }
-          if (!B_MN) {
-            tma_load_2d_pair(sB, &tmB, fbar, kb * BK, b_row0);
-          } else {
 #pragma unroll
-            for (int a = 0; a < BNH / 64; ++a)
-              tma_load_2d_pair(sB + a * kAtomBytes, &tmB, fbar, b_row0 + a * 64, kb * BK);
+          for (int acc = 0; acc < NACC; ++acc) {  // accumulator acc: tile columns acc * BN ...
+            unsigned char* sBa = sB + acc * L::B_HALF_BYTES;
+            if (!B_MN) {
+              tma_load_2d_pair(sBa, &tmB, fbar, kb * BK, b_row0 + acc * BN);
+            } else {
+#pragma unroll
+              for (int a = 0; a < BNH / 64; ++a)
+                tma_load_2d_pair(sBa + a * kAtomBytes, &tmB, fbar, b_row0 + acc * BN + a * 64,
+                                 kb * BK);
+            }
           }
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -273,8 +291,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = pair; ok && tile < n_tiles; tile += n_pairs, ++it) {
         const TileCoord c = tile_coord(p, n_m, n_n, kps, tile);
-        const int buf = it & 1;
-        const uint32_t use = (uint32_t)(it >> 1);
+        const int buf = NBUF == 2 ? (it & 1) : 0;
+        const uint32_t use = NBUF == 2 ? (uint32_t)(it >> 1) : (uint32_t)it;
+        // the second accumulator of a tile whose columns all lie past N has nothing to do
+        const int n_acc = (NACC == 2 && c.nt * TW + BN >= p.N) ? 1 : NACC;
         if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * kAccStride);
@@ -289,9 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // MN-major: step 16 rows of 128 bytes; atoms along MN are kAtomBytes apart.
             const uint64_t ad = A_MN ? umma_desc_sw128(a0 + kk * 2048, kAtomBytes, 1024)
                                      : umma_desc_sw128(a0 + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? umma_desc_sw128(b0 + kk * 2048, kAtomBytes, 1024)
-                                     : umma_desc_sw128(b0 + kk * 32, 16, 1024);
-            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int acc = 0; acc < NACC; ++acc) {
+              if (acc >= n_acc) break;
+              const uint32_t ba = b0 + acc * L::B_HALF_BYTES;
+              const uint64_t bd = B_MN ? umma_desc_sw128(ba + kk * 2048, kAtomBytes, 1024)
+                                       : umma_desc_sw128(ba + kk * 32, 16, 1024);
+              umma_bf16_pair(d_tmem + acc * BN, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+            }
           }
           umma_commit_pair_mc(&empty[stage], kPairMask);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -337,15 +362,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = pair; tile < n_tiles; tile += n_pairs, ++it) {
       const TileCoord c = tile_coord(p, n_m, n_n, kps, tile);
-      const int buf = it & 1;
-      const uint32_t use = (uint32_t)(it >> 1);
+      const int buf = NBUF == 2 ? (it & 1) : 0;
+      const uint32_t use = NBUF == 2 ? (uint32_t)(it >> 1) : (uint32_t)it;
       if (!mbar_wait(&tfull[buf], use & 1u, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kAccStride);
       const int crow0 = c.mt * 2 * BM + (int)rank * BM;  // first output row of this CTA
       const int grow = crow0 + row;  // output row (token for LSE/GRAD/DH, vocab id for DW)
       const bool row_ok = grow < p.M;
-      const int col0 = c.nt * BN;
+      const int col0 = c.nt * TW;
       const int row0 = crow0 + q * 32;  // first row of this warp's staging boxes
 
       if constexpr (KIND == TcKind::LSE) {
@@ -497,10 +522,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // fp32 partial of split c.split, plain vector stores
         float* out = p.dHp + (int64_t)c.split * p.M * p.N + (int64_t)grow * p.N;
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
+        for (int cc = 0; cc < TW / 32; ++cc) {
+          const int cb = col0 + cc * 32;
+          if (cb >= p.N && (cb - col0) % BN == 0) break;  // an accumulator past N: not computed
           float v[32];
           tmem_ld32(taddr + cc * 32, v);
-          const int cb = col0 + cc * 32;
           if (!row_ok || cb >= p.N) continue;
           if (cb + 32 <= p.N) {
             float4* dst = reinterpret_cast<float4*>(out + cb);
@@ -550,7 +576,7 @@ template <TcKind KIND>
 cudaError_t launch_kind(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
   using L = Layout<KIND>;
   const int n_m = (p.M + 2 * BM - 1) / (2 * BM);
-  const int n_n = (p.N + L::BN - 1) / L::BN;
+  const int n_n = (p.N + L::TW - 1) / L::TW;
   const int n_tiles = n_m * n_n * (KIND == TcKind::DH ? p.n_split : 1);
   if (n_tiles <= 0) return cudaSuccess;
   // The shared-memory attribute is per device: set it once per device (bit per ordinal),
@@ -599,12 +625,12 @@ cudaError_t launch_kind(const TcMaps& maps, const TcLaunch& p, cudaStream_t s) {
 
 int tc_bn(TcKind k) {
   switch (k) {
-    case TcKind::LSE: return Cfg<TcKind::LSE>::BN;
-    case TcKind::GRAD: return Cfg<TcKind::GRAD>::BN;
-    case TcKind::DH: return Cfg<TcKind::DH>::BN;
-    case TcKind::TKMAX: return Cfg<TcKind::TKMAX>::BN;
-    case TcKind::TKEMIT: return Cfg<TcKind::TKEMIT>::BN;
-    default: return Cfg<TcKind::DW>::BN;
+    case TcKind::LSE: return Layout<TcKind::LSE>::TW;
+    case TcKind::GRAD: return Layout<TcKind::GRAD>::TW;
+    case TcKind::DH: return Layout<TcKind::DH>::TW;
+    case TcKind::TKMAX: return Layout<TcKind::TKMAX>::TW;
+    case TcKind::TKEMIT: return Layout<TcKind::TKEMIT>::TW;
+    default: return Layout<TcKind::DW>::TW;
   }
 }
 

@@ -44,7 +44,7 @@ struct TcLaunch {
   unsigned* status;
   int num_sms;
 };
-int tc_bn(TcKind k);  // output tile width of a kind
+int tc_bn(TcKind k);  // output columns of one tile of a kind (all its accumulators)
 cudaError_t launch_tc(const TcMaps& maps, const TcLaunch& p, cudaStream_t s);
 
 }  // namespace ckl
