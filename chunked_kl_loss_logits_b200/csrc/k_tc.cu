@@ -60,6 +60,7 @@ constexpr int kAtomBytes = 64 * 128;  // one 64 (MN) x 64 (K) MN-major box
 constexpr int kStageBufBytes = 4096;  // one epilogue staging box: 32 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint16_t kPairMask = 0x3;
+constexpr long long kPaceMaxCycles = 1LL << 22;  // bound on the measured tile time used for pacing
 
 template <TcKind KIND>
 struct Cfg;
@@ -360,12 +361,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     int it = 0;
+    long long t_prev = 0;  // when the previous tile's accumulator became ready (SM cycles)
     for (int tile = pair; tile < n_tiles; tile += n_pairs, ++it) {
       const TileCoord c = tile_coord(p, n_m, n_n, kps, tile);
       const int buf = NBUF == 2 ? (it & 1) : 0;
       const uint32_t use = NBUF == 2 ? (uint32_t)(it >> 1) : (uint32_t)it;
       if (!mbar_wait(&tfull[buf], use & 1u, abort_flag, p.status)) break;
       tc_fence_after();
+      // The MMA time of one tile, measured as the distance between consecutive
+      // accumulators becoming ready (0 for the first tile), bounded.
+      const long long t_now = clock64();
+      const long long t_tile = t_prev > 0 ? min(t_now - t_prev, (long long)kPaceMaxCycles) : 0;
+      t_prev = t_now;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kAccStride);
       const int crow0 = c.mt * 2 * BM + (int)rank * BM;  // first output row of this CTA
       const int grow = crow0 + row;  // output row (token for LSE/GRAD/DH, vocab id for DW)
@@ -541,9 +548,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         // DW: stage 32 fp32 columns per box and add them into dW in L2
-        // (store instead of add for the first chunk).
+        // (store instead of add for the first chunk). Every pair finishes its tiles
+        // at about the same moment and each add misses L2 (dW is 2.3 GB), so
+        // issuing a whole tile's 128 KB per CTA at once floods L2 and DRAM just as
+        // the next tile's operand loads go out, and the MMA waits on them. Box group
+        // cc therefore leaves cc/10 of a tile's MMA time after the accumulator is
+        // ready (the last at 0.7 of it, well before this buffer is needed again).
 #pragma unroll 1
         for (int cc = 0; cc < BN / 32; ++cc) {
+          if (cc > 0 && t_tile > 0) {
+            const long long due = t_now + t_tile * cc / 10;
+            while (clock64() < due) __nanosleep(128);
+          }
           float v[32];
           tmem_ld32(taddr + cc * 32, v);
           const int cb = col0 + cc * 32;
