@@ -433,6 +433,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float fs = ex2_approx(m2 - ref);
 #pragma unroll 1
           for (int cc = 0; cc < BN / 64; ++cc) {
+            // the 64 KB a CTA stores per tile leave in four groups spread over the
+            // next tile's MMA time (group cc at cc/6 of it), as in the dW epilogue
+            if (cc > 0 && t_tile > 0) {
+              const long long due = t_now + t_tile * cc / 6;
+              while (clock64() < due) __nanosleep(128);
+            }
             float a[32], b[32];
             tmem_ld32(taddr + cc * 64, a);
             tmem_ld32(taddr + cc * 64 + 32, b);
