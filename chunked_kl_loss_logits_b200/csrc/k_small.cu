@@ -110,17 +110,30 @@ __global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
       if (ob > best || (ob == best && os < bslot)) { best = ob; bslot = os; }
     }
     if (bslot < K) {
+      // four 16-byte pieces of each row in flight per lane, four partial sums
       const uint4* hr = reinterpret_cast<const uint4*>(Hc + (int64_t)i * d);
       const uint4* wr = reinterpret_cast<const uint4*>(W + (int64_t)(sId[bslot] - v0) * d);
-      float z = 0.f;
-      for (int c = lane; c < (d >> 3); c += 32) {
-        const uint4 a = __ldg(hr + c), b = __ldg(wr + c);
-        z = fmaf(lo_bf16(a.x), lo_bf16(b.x), z); z = fmaf(hi_bf16(a.x), hi_bf16(b.x), z);
-        z = fmaf(lo_bf16(a.y), lo_bf16(b.y), z); z = fmaf(hi_bf16(a.y), hi_bf16(b.y), z);
-        z = fmaf(lo_bf16(a.z), lo_bf16(b.z), z); z = fmaf(hi_bf16(a.z), hi_bf16(b.z), z);
-        z = fmaf(lo_bf16(a.w), lo_bf16(b.w), z); z = fmaf(hi_bf16(a.w), hi_bf16(b.w), z);
+      const int n16 = d >> 3;
+      float zq[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int c0 = lane; c0 < n16; c0 += 128) {
+        uint4 a[4], b[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + 32 * u;
+          a[u] = c < n16 ? __ldg(hr + c) : make_uint4(0, 0, 0, 0);
+          b[u] = c < n16 ? __ldg(wr + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float z = zq[u];
+          z = fmaf(lo_bf16(a[u].x), lo_bf16(b[u].x), z); z = fmaf(hi_bf16(a[u].x), hi_bf16(b[u].x), z);
+          z = fmaf(lo_bf16(a[u].y), lo_bf16(b[u].y), z); z = fmaf(hi_bf16(a[u].y), hi_bf16(b[u].y), z);
+          z = fmaf(lo_bf16(a[u].z), lo_bf16(b[u].z), z); z = fmaf(hi_bf16(a[u].z), hi_bf16(b[u].z), z);
+          z = fmaf(lo_bf16(a[u].w), lo_bf16(b[u].w), z); z = fmaf(hi_bf16(a[u].w), hi_bf16(b[u].w), z);
+          zq[u] = z;
+        }
       }
-      r2 = warp_sum(z) * 1.4426950408889634f;
+      r2 = warp_sum((zq[0] + zq[1]) + (zq[2] + zq[3])) * 1.4426950408889634f;
     } else {
       r2 = -INFINITY;
     }

@@ -477,6 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll 1
         for (int cc = 0; cc < BN / 64; ++cc) {
+          if (cc > 0 && t_tile > 0) {  // stores spread over the next tile, as in LSE
+            const long long due = t_now + t_tile * cc / 6;
+            while (clock64() < due) __nanosleep(128);
+          }
           float a[32], b[32];
           tmem_ld32(taddr + cc * 64, a);
           tmem_ld32(taddr + cc * 64 + 32, b);
