@@ -166,6 +166,34 @@ def sampled_rows(H, W, idx, logit, rows, mask=None, with_dW=False):
     return out
 
 
+def dW_rows(H, W, idx, logit, vrows, mask=None):
+    """dW rows of the vocabulary ids `vrows`, and lse of every token (large sizes).
+
+    dW[v] = sum_t (mask_t/N) G_tv H_t with G_tv = M_t softmax(z_t)_v - P_tv (the
+    closed-form gradient of the README formula, as in fwd_bwd). Every token's
+    log-normaliser enters, so lse_t is taken over the whole vocabulary first: the
+    log-sum-exp of the log-sum-exps of blocks of W's rows (the same quantity as
+    logsumexp over all of z_t, summed in another order); G is then formed at the
+    sampled columns only. Costs O(T V d) multiply-adds and O(T) memory per block.
+    Returns (dW rows (len(vrows), d), lse (T,)).
+    """
+    H64 = np.asarray(H, dtype=F64)
+    T, V = H64.shape[0], W.shape[0]
+    block = _VBLOCK // 4
+    lse_b = []
+    for v0 in range(0, V, block):
+        lse_b.append(logsumexp(H64 @ np.asarray(W[v0:min(V, v0 + block)], dtype=F64).T))
+    lse = np.logaddexp.reduce(np.stack(lse_b, axis=1), axis=1)
+    vrows = np.asarray(vrows, dtype=np.int64)
+    p, M = teacher_probs(logit)
+    ids = np.asarray(idx, dtype=np.int64)
+    zv = H64 @ np.asarray(W[vrows], dtype=F64).T                      # T x n
+    Pv = np.stack([np.where(ids == v, p, 0.0).sum(axis=1) for v in vrows], axis=1)
+    G = M[:, None] * np.exp(zv - lse[:, None]) - Pv
+    s, _ = token_scale(mask, T)
+    return (s[:, None] * G).T @ H64, lse
+
+
 def topk_cache(H, W, K):
     """Teacher top-K cache: per token, the K largest logits of z = H W^T and their ids.
 

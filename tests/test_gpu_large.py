@@ -84,8 +84,23 @@ def test_vocab_parallel_headline_shape():
     assert rel_fro(f64(dH[rt]), r["dH"]) <= TOL["bf16"]["grad"]
     H, W, idx, logit, mask = upload(x, torch.bfloat16)
     h = ckl.ChunkedKL(w.V, w.d, w.K, max_chunk=2048)
-    l1, dH1, dW1 = h.fwd_bwd(H, W, idx, logit, mask, chunk=2048)
+    l1, dH1, dW1, lse1, _ = h.fwd_bwd(H, W, idx, logit, mask, chunk=2048, token_stats=True)
     assert rel(loss.item(), l1.item()) <= 1e-6
+    # dW rows of 64 sampled vocabulary ids (plus the most cached one) over all 4096
+    # tokens, from the oracle's log-normaliser of every token: the single-rank call
+    # (two chunks: store, then reduce-add) and the two ranks' shards
+    ids, counts = np.unique(x["idx"], return_counts=True)
+    vrows = np.unique(np.concatenate([sample_rows(w.V, 64, seed=w.seed + 5),
+                                      [ids[np.argmax(counts)]]]))
+    o_dW, o_lse = oracle.dW_rows(x["H"], x["W"], x["idx"], x["logit"], vrows, x["mask"])
+    assert float(np.max(np.abs(f64(lse1) - o_lse))) <= ROW_TOL["bf16"]["tok_abs"]
+    vt = torch.from_numpy(vrows)
+    g_dW1 = f64(dW1[vt.cuda()])
+    g_dWs = f64(torch.cat([o[2] for o in out])[vt])
+    for g in (g_dW1, g_dWs):
+        e, wr = rel_fro(g, o_dW), worst_row(g, o_dW)
+        print("vocabulary-split headline shape: dW rows", f"{e:.2e}", "worst", f"{wr:.2e}")
+        assert e <= TOL["bf16"]["grad"] and wr <= ROW_TOL["bf16"]["grad_row"]
     # the gradients of the two calls agree to within their own bf16 rounding: each
     # rank keeps its exps against a reference logit of its own rows (the single-rank
     # call against the teacher's best id), so the bf16 exps and the scaled hidden

@@ -273,6 +273,18 @@ def test_sampled_rows_match_full():
     assert rel(s_all["dW_part"], r["dW"]) <= 1e-14
 
 
+def test_dW_rows_match_full():
+    # sampled dW rows over all tokens equal the full computation's rows, and the
+    # blockwise log-normaliser equals the one over the whole row (several W blocks)
+    x = case(T=40, d=6, V=9000, K=5, seed=16, mask=True)
+    x["idx"][3, 2] = x["idx"][3, 0]  # a repeated id
+    r = oracle.fwd_bwd(x["H"], x["W"], x["idx"], x["logit"], x["mask"])
+    vrows = np.array([0, int(x["idx"][3, 0]), 4095, 4096, 8999])
+    dW, lse = oracle.dW_rows(x["H"], x["W"], x["idx"], x["logit"], vrows, x["mask"])
+    np.testing.assert_allclose(lse, r["lse"], rtol=1e-14)
+    assert rel(dW, r["dW"][vrows]) <= 1e-13
+
+
 def test_golden_fixture():
     with open(os.path.join(GOLDEN, "tiny_case.json")) as f:
         g = json.load(f)
