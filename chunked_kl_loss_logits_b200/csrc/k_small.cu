@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(
   if (lane == 0) tok[i] = make_float4(ent, cross, Msum, 0.f);
 }
 
-constexpr int kCombTok = 32, kCombSplit = 32;
+constexpr int kCombTok = 16, kCombSplit = 64;
 
 // From a token's merged (max, sum) in log2 units and its cross term: lse,
 // l_t = ent - cross + M lse and the gradient multipliers.
@@ -372,9 +372,10 @@ __device__ __forceinline__ void finish_token(int64_t t0, int i, float M2, float 
 }
 
 // Merge the per-vocabulary-tile (max, sum) partials into logsumexp(z_t), then
-// l_t = ent - cross + M lse and the gradient multipliers. A block covers 32
-// tokens; its 32 warps each merge every 32nd vocabulary tile (coalesced 256-byte
-// reads of 32 consecutive tokens), then one warp merges the 32 results.
+// l_t = ent - cross + M lse and the gradient multipliers. A block covers 16
+// tokens; its 64 thread groups of 16 each merge every 64th vocabulary tile
+// (coalesced 128-byte reads of 16 consecutive tokens), then 16 threads merge the 64
+// results (128 blocks per 2048-token chunk, so every SM takes part).
 // With `stats` set (vocabulary split over ranks) it stops at this rank's
 // (max, sum, cross) per token; vp_merge_kernel finishes after the exchange.
 __global__ void __launch_bounds__(kCombTok * kCombSplit) combine_kernel(
@@ -848,7 +849,7 @@ void launch_vp_merge(int64_t t0, int Tc, int world, int rank, const float4* stat
 
 void launch_repair(uint16_t* G, int Tc, int V, const ChunkBufs& b, int num_sms, cudaStream_t s) {
   const int n_vb = (V + 63) / 64;
-  repair_kernel<<<2 * num_sms, 256, 0, s>>>(G, n_vb, Tc, V, b.part, b.cst, b.tok, b.rep);
+  repair_kernel<<<num_sms, 256, 0, s>>>(G, n_vb, Tc, V, b.part, b.cst, b.tok, b.rep);
 }
 
 template <typename Tg>
