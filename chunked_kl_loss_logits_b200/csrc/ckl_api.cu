@@ -10,7 +10,8 @@
 //                                   (fp32: also z at the K ids and sum p z by dot products)
 //     LSE contraction               per-vocabulary-tile (max, sum exp) of z = H_c W^T and
 //                                   sum p z over the ids in the tile (bf16); stored-exp
-//                                   mode also keeps e = exp(z - tile max) in bf16
+//                                   mode also keeps E = exp(z - r) in bf16, r the row's
+//                                   reference logit (teacher kernel)
 //     combine                       lse_t, l_t, gradient multipliers
 //     stored-exp mode:  repair      rows whose stored exps used a per-tile reference
 //                                   rescaled to the row's reference R (usually none)
@@ -51,7 +52,7 @@ struct ProfRec {
 };
 
 enum KernelId {
-  KID_MASK = 0, KID_GATHER, KID_LSE, KID_COMBINE, KID_GRAD, KID_SCALE, KID_FIXUP, KID_DH,
+  KID_MASK = 0, KID_GATHER, KID_LSE, KID_COMBINE, KID_GRAD, KID_REPAIR, KID_FIXUP, KID_DH,
   KID_DH_REDUCE, KID_DW, KID_LOSS, KID_TKMAX, KID_TKTHRESH, KID_TKEMIT, KID_TKSELECT,
   KID_VP_MERGE, KID_DH_F32, KID_TO_BF16, KID_VP_GATHER, KID_VP_REDUCE, KID_COUNT
 };
@@ -424,7 +425,7 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
     if (!backward) continue;
 
     if (store_e) {
-      chk(L(KID_SCALE, 0, 0, [&] {
+      chk(L(KID_REPAIR, 0, 0, [&] {
         launch_repair(static_cast<uint16_t*>(b.G), Tc, V, b, h->num_sms, s);
       }));
     } else {
