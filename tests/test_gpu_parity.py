@@ -72,6 +72,7 @@ def test_tiny_f32_workload_full():
     (384, 192, 2048, 32, 384),    # exact multiples everywhere
     (600, 384, 5000, 20, 600),    # narrow last hidden-size tile (128 of 256 columns), 3 row tiles
     (300, 296, 2500, 8, 300),     # narrow last hidden-size tile with 40 valid columns
+    (193, 128, 2000, 16, 64),     # a last chunk of one token (dW tiles of one K-block)
 ])
 @pytest.mark.parametrize("recompute", [False, True], ids=["stored", "recompute"])
 def test_bf16_ragged_shapes(T, d, V, K, chunk, recompute):

@@ -139,6 +139,21 @@ def test_group_with_mask():
     check_against_oracle(x, out, shards)
 
 
+@pytest.mark.parametrize("rows", ["all", "half"])
+def test_group_rows_far_above_their_reference(rows):
+    # each rank keeps its exps against a reference logit of its own rows; hidden
+    # states scaled 40x put the largest logits ~100 nats above it, so the ranks'
+    # tiles fall back to their own maxima and those rows take the repair path
+    # (and rows whose cached ids all lie on other ranks take it anyway)
+    from chunked_kl_loss_logits_b200.workloads import round_to_bf16
+    x = small_case(260, 64, 2600, 12, seed=37, dtype="bf16", teacher_var=3.0, ids="zipf")
+    sel = slice(None) if rows == "all" else slice(1, None, 2)
+    x["H"][sel] *= 40.0
+    x["H"] = round_to_bf16(x["H"])
+    out, _, shards = run_group(x, 3, 100)
+    check_against_oracle(x, out, shards)
+
+
 def test_group_of_one_equals_single_rank_call():
     x = small_case(200, 128, 2000, 16, seed=32, dtype="bf16")
     out, _, _ = run_group(x, 1, 64)
