@@ -21,9 +21,11 @@
  * on the tensor cores, chunk tokens at a time, and reduced to the log-normaliser
  * in the tile's epilogue (the README's fused variant, which folds the output
  * projection into the loss and never keeps the logits of the whole sequence).
- * For the analytic gradient the default keeps exp(z - tile max) of the current
- * chunk in the chunk-bounded gradient buffer; the README's design, which forms
- * the chunk's logits again in the backward pass, is ckl_set_recompute(h, 1).
+ * For the analytic gradient the default keeps exp(z - r) of the current chunk in
+ * the chunk-bounded gradient buffer, r a per-row reference logit, and applies the
+ * one factor per row that turns it into the gradient where dH and dW are formed;
+ * the README's design, which forms the chunk's logits again in the backward pass,
+ * is ckl_set_recompute(h, 1).
  *
  * Conventions for every entry point:
  *  - All matrices are dense, row-major, contiguous. H is T x d, W is V x d,
@@ -280,10 +282,15 @@ ckl_status ckl_sync_status(ckl_handle h, void* stream);
 /* bf16 handles only: choose how the backward pass obtains exp(z - lse).
  * recompute = 1: the logits are formed a second time on the tensor cores from H
  * and W, as the README's fused variant does (executed work 8 T V d).
- * recompute = 0 (default): the forward contraction also writes exp(z - tile max)
- * in bf16 into the chunk x V gradient buffer, and the backward rescales it in
- * place (executed work 6 T V d plus one 4-byte pass over the buffer). Memory is
- * the same in both modes. fp32 handles always recompute. */
+ * recompute = 0 (default): the forward contraction also writes exp(z - r) in bf16
+ * into the chunk x V gradient buffer, r the student's logit at the token's best
+ * cached teacher id (a tile whose largest logit lies more than 2^32 above r keeps
+ * its own maximum, and its row is rescaled by a repair pass); the factor
+ * (mask/N) M exp(r - lse) is applied per row in the dH reduction and to the hidden
+ * states dW contracts with (executed work 6 T V d, no pass over the buffer). lse
+ * and the loss are the same, bit for bit, in both modes; the gradients agree to
+ * their bf16 rounding. Memory is the same in both modes. fp32 handles always
+ * recompute. */
 ckl_status ckl_set_recompute(ckl_handle h, int recompute);
 
 /* Number of kernels the handle has launched since it was created. */
