@@ -18,8 +18,12 @@
 //     recompute mode:   GRAD        G = (mask/N) M exp(z - lse), z formed again
 //     fixup                         G at the K ids: subtract (mask/N) P (stored-exp mode:
 //                                   P / (M exp(R - lse)), as G = c_t E there), in place
-//     DH contraction (+ reduce)     dH_c = G W (stored-exp: c_t (E W), and Hs = c_t H_c)
+//     DH contraction                split partials of G W (stored-exp: E W, and Hs = c_t H_c
+//                                   from the epilogue warps before their first tile)
+//       + teacher of chunk c + 1    launched behind it as a dependent (bf16 backward)
 //     DW contraction                dW (+)= G^T H_c   (stored-exp: E^T Hs; TMA reduce-add)
+//       + dH reduce                 dH_c = sum of the partials (stored-exp: times c_t),
+//                                   launched behind it as a dependent
 //   loss_finalize                   loss = sum mask l / N
 // The gradient buffer G is the only one that grows with V, and it is bounded by
 // chunk x V; everything else is O(T) or O(chunk x K).
@@ -53,12 +57,15 @@ struct ProfRec {
 
 enum KernelId {
   KID_MASK = 0, KID_GATHER, KID_LSE, KID_COMBINE, KID_GRAD, KID_REPAIR, KID_FIXUP, KID_DH,
-  KID_DH_REDUCE, KID_DW, KID_LOSS, KID_TKMAX, KID_TKTHRESH, KID_TKEMIT, KID_TKSELECT,
-  KID_VP_MERGE, KID_DH_F32, KID_TO_BF16, KID_VP_GATHER, KID_VP_REDUCE, KID_COUNT
+  KID_DW, KID_LOSS, KID_TKMAX, KID_TKTHRESH, KID_TKEMIT, KID_TKSELECT, KID_VP_MERGE,
+  KID_DH_F32, KID_TO_BF16, KID_VP_GATHER, KID_VP_REDUCE, KID_COUNT
 };
+// bf16 backward: a profiled "dh_gemm" range also holds the next chunk's teacher
+// kernel, and a "dw_gemm" range the chunk's dH split reduction, both launched
+// behind the contraction as dependents (no event may stand between the two).
 const char* kKernelNames[KID_COUNT] = {"mask_count", "teacher_topk", "lse_gemm", "lse_combine",
                                        "grad_gemm", "row_repair", "topk_fixup", "dh_gemm",
-                                       "dh_reduce", "dw_gemm", "loss_finalize", "cache_max_gemm",
+                                       "dw_gemm", "loss_finalize", "cache_max_gemm",
                                        "cache_threshold", "cache_emit_gemm", "cache_select",
                                        "vp_merge", "dh_reduce_f32", "dh_to_bf16",
                                        "vp_all_gather", "vp_all_reduce"};
@@ -334,6 +341,11 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
   chk(L(KID_MASK, 0, (double)T, [&] { launch_mask_count(mask, T, b.misc, s); }));
   if (backward && T == 0) chk(cudaMemsetAsync(dW, 0, (size_t)V * d * 4, s));
 
+  // bf16 backward: each chunk after the first has its teacher kernel launched behind
+  // the previous chunk's dH contraction, which it overlaps (it reads only that
+  // chunk's inputs and writes only per-chunk buffers the previous chunk no longer
+  // reads once its dH contraction starts).
+  bool teacher_queued = false;
   // With a group every chunk makes its two collectives even after an error (the
   // ranks' calls must stay matched); only the kernels are skipped.
   for (int64_t t0 = 0; t0 < T && (err == cudaSuccess || group); t0 += chunk) {
@@ -371,12 +383,14 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
 
     // bf16 backward keeps the exps of the forward contraction (unless recomputing)
     const bool store_e = bf16 && backward && !h->recompute;
-    if (bf16) {
+    if (bf16 && !teacher_queued) {
       chk(L(KID_GATHER, 0, (double)Tc * K * 16.0 + (store_e ? 4.0 * Tc * d : 0.0), [&] {
         launch_teacher(idx, logit, t0, Tc, V_all, v0, V, K, b, h->d_status,
                        store_e ? reinterpret_cast<const uint16_t*>(Hc) : nullptr,
-                       static_cast<const uint16_t*>(W), d, s);
+                       static_cast<const uint16_t*>(W), d, false, s);
       }));
+    } else if (bf16) {
+      teacher_queued = false;  // launched behind the previous chunk's dH contraction
     } else {
       chk(L(KID_GATHER, 2.0 * Tc * K * d, (double)Tc * (K * 8.0 + d * esz + K * d * esz), [&] {
         launch_gather<float>(static_cast<const float*>(H), static_cast<const float*>(W), idx,
@@ -462,26 +476,37 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
         continue;
       }
       mh.c = mh.a;
+      // The next chunk's teacher kernel goes behind this dH contraction (its inputs
+      // must be on the device first).
+      const int64_t t1 = t0 + chunk;
+      const int Tc1 = (int)std::min<int64_t>(chunk, T - t1);
+      const bool queue_next = t1 < T && err == cudaSuccess;
+      if (queue_next && ready) chk(cudaStreamWaitEvent(s, ready[t1 / chunk], 0));
       chk(L(KID_DH, zflops, 0, [&] {
         TcLaunch p{};
         p.kind = TcKind::DH; p.M = Tc; p.N = d; p.n_kb = (V + 63) / 64; p.n_split = P.n_split;
         p.dHp = b.dHp; p.status = h->d_status; p.num_sms = h->num_sms;
+        if (store_e) {
+          p.cst = b.cst;
+          p.Hc = reinterpret_cast<const uint16_t*>(Hc);
+          p.Hs = Hs;
+        }
         launch_tc(mh, p, s);
+        if (queue_next) {
+          // timed, when profiling, inside this record: nothing may stand between the two
+          const unsigned char* H1 = static_cast<const unsigned char*>(H) + (size_t)t1 * d * esz;
+          launch_teacher(idx, logit, t1, Tc1, V_all, v0, V, K, b, h->d_status,
+                         store_e ? reinterpret_cast<const uint16_t*>(H1) : nullptr,
+                         static_cast<const uint16_t*>(W), d, true, s);
+          h->launches++;
+          teacher_queued = true;
+        }
       }));
-      if (!group) {
-        chk(L(KID_DH_REDUCE, 0, (double)Tc * d * (4.0 * P.n_split + 2.0 + (store_e ? 4.0 : 0.0)),
-              [&] {
-          launch_dh_reduce_bf16(b.dHp, P.n_split, (int64_t)Tc * d,
-                                reinterpret_cast<uint16_t*>(dHc), d, store_e ? b.cst : nullptr,
-                                reinterpret_cast<const uint16_t*>(Hc), store_e ? Hs : nullptr, s);
-        }));
-      } else {
+      if (group) {
         // this rank's share of dH_c in fp32, summed over ranks, then bf16
-        chk(L(KID_DH_F32, 0, (double)Tc * d * (4.0 * P.n_split + 4.0 + (store_e ? 4.0 : 0.0)),
-              [&] {
+        chk(L(KID_DH_F32, 0, (double)Tc * d * (4.0 * P.n_split + 4.0), [&] {
           launch_dh_reduce_f32(b.dHp, P.n_split, (int64_t)Tc * d, dhf, d,
-                               store_e ? b.cst : nullptr, reinterpret_cast<const uint16_t*>(Hc),
-                               store_e ? Hs : nullptr, s);
+                               store_e ? b.cst : nullptr, s);
         }));
         reduce();
         chk(L(KID_TO_BF16, 0, (double)Tc * d * 6.0, [&] {
@@ -493,6 +518,13 @@ ckl_status run(ckl_ctx* h, const void* H, const void* W, const int32_t* idx, con
         p.kind = TcKind::DW; p.M = V; p.N = d; p.n_kb = (Tc + 63) / 64; p.n_split = 1;
         p.dW = dW; p.first = t0 == 0; p.status = h->d_status; p.num_sms = h->num_sms;
         launch_tc(mw, p, s);
+        if (!group) {
+          // dH_c's split reduction behind the dW contraction, in the same record
+          launch_dh_reduce_bf16(b.dHp, P.n_split, (int64_t)Tc * d,
+                                reinterpret_cast<uint16_t*>(dHc), d, store_e ? b.cst : nullptr,
+                                h->num_sms, s);
+          h->launches++;
+        }
       }));
     } else {
       const float* G = static_cast<const float*>(b.G);

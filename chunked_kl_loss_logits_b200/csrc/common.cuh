@@ -45,6 +45,39 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Stored-exp backward: the row factor c_t = gmul exp2(R - lse log2e) that turns the
+// stored exp(z - R) into the gradient (cst[t] = (lse, gmul, -, R); 0 for masked
+// tokens); 1 when there is no cst (G is the gradient itself).
+__device__ __forceinline__ float row_factor(const float4* __restrict__ cst, int64_t t) {
+  if (!cst) return 1.f;
+  const float4 q = cst[t];
+  return q.y * ex2_approx(q.w - q.x * 1.4426950408889634f);
+}
+
+// Hs[t] = bf16(c_t H[t]) for 8 elements at e8: dW then contracts the stored exps
+// with the scaled hidden states (dW = sum_t exp(z_t - R_t)^T (c_t H_t)).
+__device__ __forceinline__ void scale_h8(const uint16_t* __restrict__ Hc, uint16_t* __restrict__ Hs,
+                                         int64_t e8, float c) {
+  const uint4 x = *reinterpret_cast<const uint4*>(Hc + e8);
+  uint4 y;
+  y.x = pack_bf16x2(lo_bf16(x.x) * c, hi_bf16(x.x) * c);
+  y.y = pack_bf16x2(lo_bf16(x.y) * c, hi_bf16(x.y) * c);
+  y.z = pack_bf16x2(lo_bf16(x.z) * c, hi_bf16(x.z) * c);
+  y.w = pack_bf16x2(lo_bf16(x.w) * c, hi_bf16(x.w) * c);
+  *reinterpret_cast<uint4*>(Hs + e8) = y;
+}
+
+// ------------------------------------------------------------------ dependent launches
+// A kernel launched behind another with programmatic stream serialization may
+// start once every CTA of the one before has executed launch_dependents (or
+// exited); until then it waits like any stream-ordered launch. The waiting side's
+// griddep_wait returns once the kernel before it has completed and its writes are
+// visible; in a kernel launched the ordinary way it returns at once.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

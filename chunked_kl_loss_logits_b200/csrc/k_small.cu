@@ -12,6 +12,9 @@
 // cached entries only.
 #include <math.h>
 
+#include <algorithm>
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -40,6 +43,7 @@ __device__ __forceinline__ float dot16(const uint4& a, const uint4& b, const flo
 
 constexpr int kGatherWarps = 4;
 constexpr int kTeacherWarps = 8;
+constexpr int kReduceBlock = 512;  // dH split reduction: threads per block
 
 __host__ __device__ __forceinline__ int pow2_at_least(int k) {
   int p = 1;
@@ -60,13 +64,12 @@ __host__ __device__ __forceinline__ size_t teacher_warp_bytes(int K, int k_bytes
 // Ids are checked against the full vocabulary V_all; the sorted ids are written
 // relative to v0, the first row of this caller's slice of the LM head (0 unless
 // the vocabulary is split over ranks), so ids outside the slice match no column.
-__global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
-    const int32_t* __restrict__ idx, const float* __restrict__ logit, int64_t t0, int Tc,
-    int V_all, int v0, int V_loc, int K, int k_bytes, float4* __restrict__ tok,
-    float* __restrict__ Pk_out, int32_t* __restrict__ sid_out, float* __restrict__ sp_out,
-    unsigned* status, const uint16_t* __restrict__ Hc, const uint16_t* __restrict__ W, int d,
-    int* __restrict__ rep) {
-  extern __shared__ __align__(16) unsigned char smem[];
+__device__ __forceinline__ void teacher_token(
+    unsigned char* smem, const int32_t* __restrict__ idx, const float* __restrict__ logit,
+    int64_t t0, int Tc, int V_all, int v0, int V_loc, int K, int k_bytes,
+    float4* __restrict__ tok, float* __restrict__ Pk_out, int32_t* __restrict__ sid_out,
+    float* __restrict__ sp_out, unsigned* status, const uint16_t* __restrict__ Hc,
+    const uint16_t* __restrict__ W, int d, int* __restrict__ rep) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * kTeacherWarps + warp;
   if (rep && blockIdx.x == 0 && threadIdx.x == 0) rep[0] = 0;  // this chunk's repair list
@@ -204,6 +207,23 @@ __global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
   ent = warp_sum(ent);
   Msum = warp_sum(Msum);
   if (lane == 0) tok[i] = make_float4(ent, 0.f, Msum, r2);
+}
+
+// The next chunk's teacher statistics may run behind the current chunk's dH
+// contraction as a dependent launch (two blocks beside each of its CTAs); they
+// touch none of that kernel's inputs or outputs. One thread then waits for the dH
+// kernel to complete, so that this kernel's completion still orders the dW
+// contraction and everything after it behind both.
+__global__ void __launch_bounds__(kTeacherWarps * 32) teacher_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ logit, int64_t t0, int Tc,
+    int V_all, int v0, int V_loc, int K, int k_bytes, float4* __restrict__ tok,
+    float* __restrict__ Pk_out, int32_t* __restrict__ sid_out, float* __restrict__ sp_out,
+    unsigned* status, const uint16_t* __restrict__ Hc, const uint16_t* __restrict__ W, int d,
+    int* __restrict__ rep) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  teacher_token(smem, idx, logit, t0, Tc, V_all, v0, V_loc, K, k_bytes, tok, Pk_out, sid_out,
+                sp_out, status, Hc, W, d, rep);
+  if (blockIdx.x == 0 && threadIdx.x == 0) griddep_wait();
 }
 
 // One warp per token of the chunk.
@@ -527,31 +547,10 @@ __global__ void fixup_kernel(const int32_t* __restrict__ idx, int64_t t0, int Tc
 }
 
 // Sum of the split-K partials in fp32 (vocabulary split over ranks: the ranks'
-// sums are added by the exchange before the conversion to bf16).
-// Stored-exp backward: the row factor c_t = gmul exp2(R - lse log2e) that turns the
-// stored exp(z - R) into the gradient (0 for masked tokens); 1 when G is the gradient.
-__device__ __forceinline__ float row_factor(const float4* __restrict__ cst, int64_t t) {
-  if (!cst) return 1.f;
-  const float4 q = cst[t];
-  return q.y * ex2_approx(q.w - q.x * 1.4426950408889634f);
-}
-
-// Hs[t] = bf16(c_t H[t]) for 8 elements at e8: DW then contracts the stored exps
-// with the scaled hidden states (dW = sum_t exp(z_t - R_t)^T (c_t H_t)).
-__device__ __forceinline__ void scale_h8(const uint16_t* __restrict__ Hc, uint16_t* __restrict__ Hs,
-                                         int64_t e8, float c) {
-  const uint4 x = *reinterpret_cast<const uint4*>(Hc + e8);
-  uint4 y;
-  y.x = pack_bf16x2(lo_bf16(x.x) * c, hi_bf16(x.x) * c);
-  y.y = pack_bf16x2(lo_bf16(x.y) * c, hi_bf16(x.y) * c);
-  y.z = pack_bf16x2(lo_bf16(x.z) * c, hi_bf16(x.z) * c);
-  y.w = pack_bf16x2(lo_bf16(x.w) * c, hi_bf16(x.w) * c);
-  *reinterpret_cast<uint4*>(Hs + e8) = y;
-}
-
+// sums are added by the exchange before the conversion to bf16); each row times
+// its row factor (1 without cst).
 __global__ void dh_reduce_f32_kernel(const float* __restrict__ dHp, int n_split, int64_t n_elem,
-                                     float* __restrict__ out, int d, const float4* __restrict__ cst,
-                                     const uint16_t* __restrict__ Hc, uint16_t* __restrict__ Hs) {
+                                     float* __restrict__ out, int d, const float4* __restrict__ cst) {
   const int64_t e8 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (e8 >= n_elem) return;
   float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -565,7 +564,6 @@ __global__ void dh_reduce_f32_kernel(const float* __restrict__ dHp, int n_split,
   float4* o = reinterpret_cast<float4*>(out + e8);
   o[0] = make_float4(a[0] * c, a[1] * c, a[2] * c, a[3] * c);
   o[1] = make_float4(a[4] * c, a[5] * c, a[6] * c, a[7] * c);
-  if (Hs) scale_h8(Hc, Hs, e8, c);
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ in, int64_t n_elem,
@@ -579,31 +577,37 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ in, int64_t n_elem,
   *reinterpret_cast<uint2*>(out + e4) = o;
 }
 
-__global__ void dh_reduce_bf16_kernel(const float* __restrict__ dHp, int n_split, int64_t n_elem,
-                                      uint16_t* __restrict__ dH, int d,
-                                      const float4* __restrict__ cst,
-                                      const uint16_t* __restrict__ Hc, uint16_t* __restrict__ Hs) {
-  const int64_t e8 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
-  if (e8 >= n_elem) return;
-  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < n_split; ++s) {
-    const float4* p = reinterpret_cast<const float4*>(dHp + s * n_elem + e8);
-    const float4 x = p[0], y = p[1];
-    a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
-    a[4] += y.x; a[5] += y.y; a[6] += y.z; a[7] += y.w;
-  }
-  const float c = row_factor(cst, e8 / d);
-  if (cst) {
+// Sum of the split-K partials -> bf16 dH, each row times its row factor, over a
+// grid that strides the chunk (one block per SM). It may run behind the dW
+// contraction as a dependent launch (one block beside each of that kernel's CTAs):
+// one thread then waits for the dW kernel to complete, so this kernel's completion
+// still orders everything after it behind both.
+__global__ void __launch_bounds__(kReduceBlock) dh_reduce_bf16_kernel(
+    const float* __restrict__ dHp, int n_split, int64_t n_elem, uint16_t* __restrict__ dH, int d,
+    const float4* __restrict__ cst) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x * 8;
+  for (int64_t e8 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; e8 < n_elem;
+       e8 += stride) {
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < n_split; ++s) {
+      const float4* p = reinterpret_cast<const float4*>(dHp + s * n_elem + e8);
+      const float4 x = p[0], y = p[1];
+      a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
+      a[4] += y.x; a[5] += y.y; a[6] += y.z; a[7] += y.w;
+    }
+    if (cst) {
+      const float c = row_factor(cst, e8 / d);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] *= c;
+      for (int k = 0; k < 8; ++k) a[k] *= c;
+    }
+    uint4 o;
+    o.x = pack_bf16x2(a[0], a[1]);
+    o.y = pack_bf16x2(a[2], a[3]);
+    o.z = pack_bf16x2(a[4], a[5]);
+    o.w = pack_bf16x2(a[6], a[7]);
+    *reinterpret_cast<uint4*>(dH + e8) = o;
   }
-  if (Hs) scale_h8(Hc, Hs, e8, c);
-  uint4 o;
-  o.x = pack_bf16x2(a[0], a[1]);
-  o.y = pack_bf16x2(a[2], a[3]);
-  o.z = pack_bf16x2(a[4], a[5]);
-  o.w = pack_bf16x2(a[6], a[7]);
-  *reinterpret_cast<uint4*>(dH + e8) = o;
+  if (blockIdx.x == 0 && threadIdx.x == 0) griddep_wait();
 }
 
 // ------------------------------------------------------------ teacher top-K cache
@@ -796,6 +800,20 @@ __global__ void __launch_bounds__(kReduceThreads) loss_finalize_kernel(
 
 inline unsigned blocks_for(int64_t n, int per) { return (unsigned)((n + per - 1) / per); }
 
+// A kernel that runs beside the tensor-core kernels (as a dependent launch) asks for
+// their shared-memory split, so an SM need not change it to take the kernel's
+// blocks. Set once per device (`done`: one bit per device ordinal).
+template <typename Kernel>
+void prefer_max_shared(Kernel fn, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) == cudaSuccess)
+    done.fetch_or(bit, std::memory_order_release);
+}
+
 }  // namespace
 
 void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t s) {
@@ -804,14 +822,25 @@ void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t 
 
 void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V_all, int v0,
                     int V_loc, int K, const ChunkBufs& b, unsigned* status, const uint16_t* Hc,
-                    const uint16_t* W, int d, cudaStream_t s) {
+                    const uint16_t* W, int d, bool behind, cudaStream_t s) {
   const int k_bytes = (K * 4 + 15) & ~15;
   const size_t smem = (size_t)kTeacherWarps * teacher_warp_bytes(K, k_bytes);
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(teacher_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  teacher_kernel<<<blocks_for(Tc, kTeacherWarps), kTeacherWarps * 32, smem, s>>>(
-      idx, logit, t0, Tc, V_all, v0, V_loc, K, k_bytes, b.tok, b.Pk, b.sid, b.sp, status, Hc, W,
-      d, Hc ? b.rep : nullptr);
+  static std::atomic<uint64_t> carveout_set{0};
+  prefer_max_shared(teacher_kernel, carveout_set);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks_for(Tc, kTeacherWarps));
+  cfg.blockDim = dim3(kTeacherWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = behind ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, teacher_kernel, idx, logit, t0, Tc, V_all, v0, V_loc, K, k_bytes, b.tok,
+                     b.Pk, b.sid, b.sp, status, Hc, W, d, Hc ? b.rep : nullptr);
 }
 
 template <typename Tin>
@@ -864,15 +893,27 @@ template void launch_fixup<uint16_t>(const int32_t*, int64_t, int, int, int, int
                                      const ChunkBufs&, bool, cudaStream_t);
 
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH, int d,
-                           const float4* cst, const uint16_t* Hc, uint16_t* Hs, cudaStream_t s) {
-  dh_reduce_bf16_kernel<<<blocks_for(n_elem / 8, 256), 256, 0, s>>>(dHp, n_split, n_elem, dH, d,
-                                                                    cst, Hc, Hs);
+                           const float4* cst, int num_sms, cudaStream_t s) {
+  const int64_t need = (n_elem / 8 + kReduceBlock - 1) / kReduceBlock;
+  static std::atomic<uint64_t> carveout_set{0};
+  prefer_max_shared(dh_reduce_bf16_kernel, carveout_set);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(need, num_sms)));
+  cfg.blockDim = dim3(kReduceBlock);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, dh_reduce_bf16_kernel, dHp, n_split, n_elem, dH, d, cst);
 }
 
 void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out, int d,
-                          const float4* cst, const uint16_t* Hc, uint16_t* Hs, cudaStream_t s) {
+                          const float4* cst, cudaStream_t s) {
   dh_reduce_f32_kernel<<<blocks_for(n_elem / 8, 256), 256, 0, s>>>(dHp, n_split, n_elem, out, d,
-                                                                   cst, Hc, Hs);
+                                                                   cst);
 }
 
 void launch_f32_to_bf16(const float* in, int64_t n_elem, uint16_t* out, cudaStream_t s) {

@@ -223,6 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();  // barriers of both CTAs initialised before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Every CTA of this persistent grid is resident: a kernel launched behind this one
+  // as a dependent may take what room is left on the SMs from here on.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -360,6 +363,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++nstage;
     };
 
+    if constexpr (KIND == TcKind::DH) {
+      // The scaled hidden states the dW contraction reads, written while these warps
+      // would otherwise wait for their first accumulator (~a millisecond away).
+      if (p.Hs) {
+        const int64_t n8 = (int64_t)p.M * p.N / 8;
+        const int64_t step = (int64_t)gridDim.x * 128;
+        for (int64_t e = (int64_t)blockIdx.x * 128 + (threadIdx.x - 64); e < n8; e += step)
+          scale_h8(p.Hc, p.Hs, e * 8, row_factor(p.cst, e * 8 / p.N));
+      }
+    }
     int it = 0;
     long long t_prev = 0;  // when the previous tile's accumulator became ready (SM cycles)
     for (int tile = pair; tile < n_tiles; tile += n_pairs, ++it) {

@@ -28,10 +28,14 @@ struct TcLaunch {
                    // row's reference tok[row].w (log2 units), or the tile's maximum when
                    // that lies more than kRefGap above it
   const float4* tok;  // LSE with store_e: per-row values, .w = the reference
-  const float4* cst;  // GRAD
+  const float4* cst;  // GRAD; DH with Hs (row factors)
   uint16_t* G;        // GRAD
   int64_t ldG;        // GRAD
   float* dHp;         // DH
+  // DH, stored-exp backward: the epilogue warps also write Hs = bf16(c_t Hc) (M x N,
+  // c_t the row factor from cst) for the dW contraction, before their first tile
+  const uint16_t* Hc;
+  uint16_t* Hs;
   float* dW;          // DW
   int first;          // DW: overwrite instead of accumulate
   // teacher top-K cache: TKMAX writes each row's best (logit, id) per vocabulary

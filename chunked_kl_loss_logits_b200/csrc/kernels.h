@@ -47,10 +47,12 @@ void launch_mask_count(const uint8_t* mask, int64_t T, Misc* misc, cudaStream_t 
 // over ranks: this rank holds rows [v0, v0 + V_loc) of W; otherwise v0 = 0,
 // V_all = V_loc). With Hc (the chunk's hidden states; W and d then too): also the
 // reference logit r2 of the stored-exp backward into tok.w, and the chunk's
-// repair list is emptied.
+// repair list is emptied. behind: launched as a dependent of the kernel just
+// enqueued on s (the previous chunk's dH contraction), which it may overlap; its
+// completion still implies that kernel's.
 void launch_teacher(const int32_t* idx, const float* logit, int64_t t0, int Tc, int V_all, int v0,
                     int V_loc, int K, const ChunkBufs& b, unsigned* status, const uint16_t* Hc,
-                    const uint16_t* W, int d, cudaStream_t s);
+                    const uint16_t* W, int d, bool behind, cudaStream_t s);
 // fp32: as launch_teacher, plus the student logits at the ids by dot products.
 template <typename Tin>
 void launch_gather(const Tin* H, const Tin* W, const int32_t* idx, const float* logit, int64_t t0,
@@ -76,10 +78,11 @@ void launch_fixup(const int32_t* idx, int64_t t0, int Tc, int K, int V, int v0, 
 // reference R, in place (G blocked, bf16); nothing to do for an empty list.
 void launch_repair(uint16_t* G, int Tc, int V, const ChunkBufs& b, int num_sms, cudaStream_t s);
 // Sum of the n_split partials of dH_c -> bf16 dH. With cst (stored-exp backward)
-// each row is multiplied by c_t = gmul exp(R - lse), and Hs = bf16(c_t Hc) is written
-// for the dW contraction (Hs may be NULL).
+// each row is multiplied by c_t = gmul exp(R - lse). Launched as a dependent of the
+// kernel just enqueued on s (the chunk's dW contraction), which it overlaps on at
+// most num_sms blocks; its completion still implies that kernel's.
 void launch_dh_reduce_bf16(const float* dHp, int n_split, int64_t n_elem, uint16_t* dH, int d,
-                           const float4* cst, const uint16_t* Hc, uint16_t* Hs, cudaStream_t s);
+                           const float4* cst, int num_sms, cudaStream_t s);
 // One thread waits on a barrier nothing arrives at until the wait bound fires.
 void launch_wait_selftest(unsigned* status, long long* cycles, cudaStream_t s);
 // Top-K cache with the vocabulary split over ranks: pack this rank's K best as
@@ -89,9 +92,9 @@ void launch_topk_pack(const int32_t* idx, const float* lg, int64_t n, int v0, fl
 void launch_topk_regroup(const float2* gathered, int world, int rows, int K, float2* cand, int* cnt,
                          cudaStream_t s);
 // As launch_dh_reduce_bf16 with an fp32 result (the vocabulary-parallel all-reduce's
-// buffer). n_elem % 8 == 0.
+// buffer), launched the ordinary way. n_elem % 8 == 0.
 void launch_dh_reduce_f32(const float* dHp, int n_split, int64_t n_elem, float* out, int d,
-                          const float4* cst, const uint16_t* Hc, uint16_t* Hs, cudaStream_t s);
+                          const float4* cst, cudaStream_t s);
 void launch_f32_to_bf16(const float* in, int64_t n_elem, uint16_t* out, cudaStream_t s);
 // Teacher top-K cache: per row, the threshold = the K-th best of the n_vt tile
 // bests (logit descending, id ascending), or "take everything" when n_vt <= K.

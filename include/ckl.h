@@ -287,7 +287,8 @@ ckl_status ckl_sync_status(ckl_handle h, void* stream);
  * cached teacher id (a tile whose largest logit lies more than 2^32 above r keeps
  * its own maximum, and its row is rescaled by a repair pass); the factor
  * (mask/N) M exp(r - lse) is applied per row in the dH reduction and to the hidden
- * states dW contracts with (executed work 6 T V d, no pass over the buffer). lse
+ * states dW contracts with (a scaled copy the dH contraction writes; executed work
+ * 6 T V d, no pass over the buffer). lse
  * and the loss are the same, bit for bit, in both modes; the gradients agree to
  * their bf16 rounding. Memory is the same in both modes. fp32 handles always
  * recompute. */
@@ -298,7 +299,11 @@ int64_t ckl_launch_count(ckl_handle h);
 
 /* Per-kernel timing. When enabled, each kernel launch is bracketed by CUDA
  * events on the launching stream (a pool of `max_launches` event pairs is
- * created here; launches past that are not timed). */
+ * created here; launches past that are not timed). Two kernels of the bf16
+ * backward run behind a contraction as dependent launches and are timed inside
+ * its range: the next chunk's teacher kernel inside "dh_gemm", the chunk's dH
+ * split reduction inside "dw_gemm" (an event between the two launches would
+ * serialise them). */
 ckl_status ckl_profile_enable(ckl_handle h, int enable, int max_launches);
 
 typedef struct {
