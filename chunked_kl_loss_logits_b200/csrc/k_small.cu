@@ -585,27 +585,58 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ in, int64_t n_elem,
 __global__ void __launch_bounds__(kReduceBlock) dh_reduce_bf16_kernel(
     const float* __restrict__ dHp, int n_split, int64_t n_elem, uint16_t* __restrict__ dH, int d,
     const float4* __restrict__ cst) {
+  // Per thread and round: U groups of 8 elements; the partials of up to SG splits are
+  // loaded together before they are added (in split order). U = 1 keeps a block within
+  // the registers the dW contraction's CTA leaves on its SM.
+  constexpr int U = 1, SG = 4;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x * 8;
-  for (int64_t e8 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; e8 < n_elem;
-       e8 += stride) {
-    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < n_split; ++s) {
-      const float4* p = reinterpret_cast<const float4*>(dHp + s * n_elem + e8);
-      const float4 x = p[0], y = p[1];
-      a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
-      a[4] += y.x; a[5] += y.y; a[6] += y.z; a[7] += y.w;
-    }
-    if (cst) {
-      const float c = row_factor(cst, e8 / d);
+  for (int64_t e0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; e0 < n_elem;
+       e0 += U * stride) {
+    float a[U][8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) a[k] *= c;
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) a[u][k] = 0.f;
+    for (int s0 = 0; s0 < n_split; s0 += SG) {
+      float4 x[SG][U], y[SG][U];
+#pragma unroll
+      for (int g = 0; g < SG; ++g)
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int64_t e8 = e0 + u * stride;
+          x[g][u] = y[g][u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (s0 + g < n_split && e8 < n_elem) {
+            const float4* p = reinterpret_cast<const float4*>(dHp + (s0 + g) * n_elem + e8);
+            x[g][u] = p[0];
+            y[g][u] = p[1];
+          }
+        }
+#pragma unroll
+      for (int g = 0; g < SG; ++g)
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          if (s0 + g < n_split) {
+            a[u][0] += x[g][u].x; a[u][1] += x[g][u].y; a[u][2] += x[g][u].z; a[u][3] += x[g][u].w;
+            a[u][4] += y[g][u].x; a[u][5] += y[g][u].y; a[u][6] += y[g][u].z; a[u][7] += y[g][u].w;
+          }
+        }
     }
-    uint4 o;
-    o.x = pack_bf16x2(a[0], a[1]);
-    o.y = pack_bf16x2(a[2], a[3]);
-    o.z = pack_bf16x2(a[4], a[5]);
-    o.w = pack_bf16x2(a[6], a[7]);
-    *reinterpret_cast<uint4*>(dH + e8) = o;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t e8 = e0 + u * stride;
+      if (e8 >= n_elem) continue;
+      if (cst) {
+        const float c = row_factor(cst, e8 / d);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a[u][k] *= c;
+      }
+      uint4 o;
+      o.x = pack_bf16x2(a[u][0], a[u][1]);
+      o.y = pack_bf16x2(a[u][2], a[u][3]);
+      o.z = pack_bf16x2(a[u][4], a[u][5]);
+      o.w = pack_bf16x2(a[u][6], a[u][7]);
+      *reinterpret_cast<uint4*>(dH + e8) = o;
+    }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) griddep_wait();
 }
