@@ -204,6 +204,32 @@ def test_chunk_invariance():
         assert rel_fro(cur[2], ref[2]) <= 1e-5
 
 
+@pytest.mark.parametrize("recompute", [False, True], ids=["stored", "recompute"])
+def test_many_short_chunks(recompute):
+    # 8- and 16-token chunks: every kernel of a chunk is short, so the next chunk's
+    # teacher kernel (launched behind the dH contraction) and the dH reduction
+    # (behind the dW contraction) overlap as much of their neighbours as they can;
+    # the results must equal the one-chunk call (lse and l_t bit for bit) and the oracle
+    x = small_case(300, 64, 1200, 16, seed=31, dtype="bf16", teacher_var=3.0, ids="zipf",
+                   packing=True)
+    H, W, idx, logit, mask = upload(x, torch.bfloat16)
+    h = ckl.ChunkedKL(1200, 64, 16, max_chunk=300)
+    h.set_recompute(recompute)
+    ref = h.fwd_bwd(H, W, idx, logit, mask, chunk=300, token_stats=True)
+    r = oracle.fwd_bwd(x["H"], x["W"], x["idx"], x["logit"], x["mask"])
+    for chunk in (16, 8):
+        loss, dH, dW, lse, ell = h.fwd_bwd(H, W, idx, logit, mask, chunk=chunk, token_stats=True)
+        h.sync_status()
+        assert torch.equal(lse, ref[3]) and torch.equal(ell, ref[4])
+        assert rel(loss.item(), ref[0].item()) <= 1e-6
+        assert rel_fro(f64(dW), f64(ref[2])) <= 1e-5
+        assert rel_fro(f64(dH), f64(ref[1])) <= 1e-3
+        assert rel(loss.item(), r["loss"]) <= TOL["bf16"]["loss"]
+        assert rel_fro(f64(dH), r["dH"]) <= TOL["bf16"]["grad"]
+        assert rel_fro(f64(dW), r["dW"]) <= TOL["bf16"]["grad"]
+    h.close()
+
+
 def test_forward_only_matches_fused_loss():
     x = small_case(260, 64, 1000, 16, seed=17, dtype="bf16")
     H, W, idx, logit, mask = upload(x, torch.bfloat16)
