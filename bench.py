@@ -213,6 +213,10 @@ def oracle_rate(x, w, steps: int = 1, warmup: int = 1):
     cores = max([i.get("num_threads", 1) for i in info] + [1])
     W64 = np.asarray(x["W"], dtype=np.float64)  # untimed, once
     n_a, n_b = ORACLE_ROWS
+    # one untimed call first: starting the BLAS threads and touching fresh pages are
+    # not per-token costs, whatever the warm-up count
+    oracle.sampled_rows(x["H"], W64, x["idx"], x["logit"], np.arange(min(n_a, w.T)), x["mask"],
+                        with_dW=True)
     rates, fixed = [], []
     for s in range(warmup + steps):
         t_call = []
@@ -222,18 +226,31 @@ def oracle_rate(x, w, steps: int = 1, warmup: int = 1):
             t0 = time.perf_counter()
             oracle.sampled_rows(x["H"], W64, x["idx"], x["logit"], rows, x["mask"], with_dW=True)
             t_call.append(time.perf_counter() - t0)
-        per_tok = max(t_call[1] - t_call[0], 1e-9) / (n_b - n_a)
+        if t_call[1] > t_call[0]:
+            per_tok = (t_call[1] - t_call[0]) / (n_b - n_a)
+            fix = t_call[0] - n_a * per_tok
+        else:
+            # the fixed cost swamps the per-token one (a small vocabulary) and the two
+            # times do not order: the larger call's whole time per token, a lower rate
+            per_tok = t_call[1] / n_b
+            fix = float("nan")
         if s >= warmup:
             rates.append(1.0 / per_tok)
-            fixed.append(t_call[0] - n_a * per_tok)
+            fixed.append(fix)
     return rates, fixed, (n_a, n_b), cores
 
 
 def oracle_sample_text(rows, steps, fixed):
-    return (f"slope of two oracle calls per step ({rows[0]} and {rows[1]} consecutive tokens of the "
+    slopes = [f for f in fixed if f == f]  # NaN marks a step timed by its whole call
+    text = (f"slope of two oracle calls per step ({rows[0]} and {rows[1]} consecutive tokens of the "
             f"workload; full per-token path: lse, l_t, dH row, dW share; fp64 numpy/BLAS, W widened "
-            f"to fp64 once before timing), {steps} timed step(s); per-call fixed cost "
-            f"{statistics.median(fixed):.2f} s excluded")
+            f"to fp64 once before timing), {steps} timed step(s)")
+    if slopes:
+        text += f"; per-call fixed cost {statistics.median(slopes):.2f} s excluded"
+    if len(slopes) < len(fixed):
+        text += (f"; {len(fixed) - len(slopes)} step(s) whose two times did not order timed by the "
+                 f"{rows[1]}-token call's whole time, fixed cost included")
+    return text
 
 
 def bench_config(w, mask, chunk, recompute, world):
