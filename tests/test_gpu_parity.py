@@ -230,6 +230,33 @@ def test_many_short_chunks(recompute):
     h.close()
 
 
+def test_two_handles_on_two_streams():
+    # two calls in flight at once, each on its own handle, workspace and stream: any
+    # kernel of one call (the dependent launches included) may run beside the other's;
+    # each result must equal the same call made alone, bit for bit
+    dev = torch.device("cuda", 0)
+    xs = [small_case(600, 128, 3000, 16, seed=s, dtype="bf16", teacher_var=3.0, ids="zipf",
+                     packing=True) for s in (61, 62)]
+    ins = [upload(x, torch.bfloat16) for x in xs]
+    hs = [ckl.ChunkedKL(3000, 128, 16, max_chunk=128, device=dev) for _ in xs]
+    refs = [h.fwd_bwd(*i, chunk=128) for h, i in zip(hs, ins)]
+    wss = [h.workspace(600, 128) for h in hs]
+    outs = [(torch.empty((), device=dev), torch.empty_like(i[0]),
+             torch.empty((3000, 128), dtype=torch.float32, device=dev)) for i in ins]
+    streams = [torch.cuda.Stream(dev) for _ in xs]
+    torch.cuda.synchronize(dev)
+    for _ in range(3):
+        for h, i, o, ws, st in zip(hs, ins, outs, wss, streams):
+            h.fwd_bwd(*i, chunk=128, out=o, workspace=ws, sync=False, stream=st)
+        torch.cuda.synchronize(dev)
+        for h, o, r in zip(hs, outs, refs):
+            h.sync_status()
+            for a, b in zip(o, r):
+                assert torch.equal(a, b)
+    for h in hs:
+        h.close()
+
+
 def test_forward_only_matches_fused_loss():
     x = small_case(260, 64, 1000, 16, seed=17, dtype="bf16")
     H, W, idx, logit, mask = upload(x, torch.bfloat16)
