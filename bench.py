@@ -112,12 +112,23 @@ KERNEL_SOURCES = ("chunked_kl_loss_logits_b200/csrc/k_tc.cu", "chunked_kl_loss_l
                   "chunked_kl_loss_logits_b200/csrc/k_tc.h")
 
 
-def kernel_source_hash() -> str:
+def code_text(src: str) -> str:
+    """C++/CUDA source without its comments and with whitespace runs collapsed: the
+    text that decides what the compiler builds (string literals hold no comment
+    markers in these files)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
+def kernel_source_hash(root: str = ROOT) -> str:
+    """Hash of the tensor-core kernels' code (comments and layout excluded)."""
     import hashlib
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(root, rel), encoding="utf-8") as f:
+            h.update(code_text(f.read()).encode())
     return h.hexdigest()[:16]
 
 

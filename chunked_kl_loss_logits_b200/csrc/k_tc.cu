@@ -34,14 +34,15 @@
 //   warp 1      allocates 512 TMEM columns in both CTAs; in the even CTA one
 //               thread issues the pair MMAs (M=256, N=256, K=16) into one of two
 //               accumulators and commits each stage to the `empty` barriers of
-//               both CTAs (tcgen05.commit multicast).
+//               both CTAs (one tcgen05.commit arriving in both).
 //   warps 2..5  epilogue (both CTAs): tcgen05.ld of the CTA's 128 accumulator
 //               rows (thread = row), the kind's math, plain stores or 128B-swizzled
 //               staging + TMA bulk stores, then one arrival per warp on the even
 //               CTA's `tempty` barrier.
 // Operand layouts: H, W and G are read K-major for LSE/GRAD/DH-A; W (DH-B), G
 // (DW-A) and H (DW-B) are read MN-major, so no operand is ever transposed in
-// memory. No load uses cluster multicast. Every wait is bounded (common.cuh).
+// memory. Every TMA load fills the issuing CTA's own shared memory only. Every
+// wait is bounded (common.cuh).
 #include <atomic>
 
 #include "common.cuh"

@@ -49,3 +49,9 @@ def test_reference_arm_json_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_kernel_hash_ignores_comments_and_layout():
+    # the recorded DRAM traffic is keyed to the kernels' code, not to their comments
+    assert bench.code_text("int a; // note\n/* block\n comment */  int  b;\n") == "int a; int b;"
+    assert bench.code_text('asm("ex2.approx.f32 %0, %1;");') == 'asm("ex2.approx.f32 %0, %1;");'
