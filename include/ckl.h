@@ -137,8 +137,8 @@ ckl_status ckl_fwd_bwd_from_host(ckl_handle h, const void* H_host, const int32_t
 /* Forward-only loss that allocates nothing, for callers that may not call
  * cudaMalloc: code embedded in a runtime that owns all device memory through its
  * own arena or caching allocator, and latency-critical loops that cannot afford
- * the device-wide synchronisation of cudaMalloc / cudaFree. (The paper and its
- * pages have no counterpart: this is a deployment variant of ckl_forward.)
+ * the device-wide synchronisation of cudaMalloc / cudaFree. (The source pages
+ * have no counterpart: this is a deployment variant of ckl_forward.)
  * No handle is involved, since ckl_create allocates. The forward workspace and
  * the device status word live in one file-scope device array of 32 MiB that
  * every GPU which loads this library keeps until the process exits. A call whose
